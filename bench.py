@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A16 MoE layer (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--path PATH]
+                    [--impl ours|reference]
+
+Default workload (the one the tokens/s metric is quoted on): OLMoE-shaped decode, 16 layers of
+H=2048, I=1024, E=64 experts all resident, top-8, one token per step, fresh router logits
+every step. A step is one token through all 16 layers: for every layer the router, grouping,
+gate/up with SiLU*up, down projection and combine (the packer runs offline, before timing).
+Weights are drawn on the device (seeded), packed once by the library's packer and stay
+resident; per-step activations and logits are pre-generated and resident. The 3.3 GB packed
+bank and the per-step routing keep every layer's experts out of L2 between reuses ("inputs
+larger than L2").
+
+value: tokens/s over all ranks (each rank runs its own replica: the layer does not shard
+across GPUs here), timed with CUDA events around exactly K steps, max over ranks.
+e2e: the same steps through the same C ABI with the per-step inputs copied from pinned host
+memory and every layer's output copied back, host synchronising on each step.
+roofline: the dominant kernel's algorithmic bytes (distinct routed experts' packed weights and
+scales) per launch over its CUDA-event duration, against the measured HBM copy bandwidth.
+cpu_baseline: the oracle (plain C++) on the host cores over a bounded sample of the workload.
+--impl reference times that oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "W4A16 MoE-layer tokens/s; % of HBM roofline (decode) / tensor peak (prefill)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def expert_bytes(H: int, I: int) -> int:
+    codes = 2 * I * H // 2 + H * I // 2
+    scales = 2 * (2 * I * (H // 128) + H * (I // 128))
+    return codes + scales
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(parts)
+            except ValueError:
+                pass
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if (args.impl == "ours" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def all_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+class OracleLayer:
+    """One layer of the workload packed by the oracle on the host (CPU baseline / reference)."""
+
+    def __init__(self, wl: mi.Workload, layer: int, experts):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.w13 = np.zeros((wl.E, oracle.packed_bytes(2 * wl.I, wl.H)), np.uint8)
+        self.s13 = np.zeros((wl.E, oracle.scale_count(2 * wl.I, wl.H)), np.uint16)
+        self.w2 = np.zeros((wl.E, oracle.packed_bytes(wl.H, wl.I)), np.uint8)
+        self.s2 = np.zeros((wl.E, oracle.scale_count(wl.H, wl.I)), np.uint16)
+        for e in experts:
+            a, b = mi.expert_weights(wl, layer, e)
+            self.w13[e], self.s13[e] = oracle.pack(*oracle.quantize(a))
+            self.w2[e], self.s2[e] = oracle.pack(*oracle.quantize(b))
+
+    def forward(self, x, logits, threads: int):
+        idx, wts = self.oracle.route(logits, self.wl.k)
+        return self.oracle.moe_ffn(x, idx, wts, self.w13, self.s13, self.w2, self.s2, self.wl.H, self.wl.I,
+                                   n_threads=threads)
+
+
+def oracle_threads(wl: mi.Workload) -> int:
+    return max(1, min(os.cpu_count() or 1, wl.T * wl.k))
+
+
+def cpu_baseline(wl: mi.Workload, budget_s: float = 12.0):
+    """Oracle tokens/s over a bounded sample: one layer (the routed experts of one logits draw,
+    packed by the oracle), forwards repeated for about budget_s, scaled by the layer count."""
+    logits = mi.router_logits(wl, 0, 0)
+    import oracle
+    idx, _ = oracle.route(logits, wl.k)
+    layer = OracleLayer(wl, 0, sorted(set(idx.ravel().tolist())))
+    x = mi.activations(wl, 0, 0)
+    threads = oracle_threads(wl)
+    layer.forward(x, logits, threads)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        layer.forward(x, logits, threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 1000:
+            break
+    per_layer = el / reps
+    value = wl.T / (per_layer * wl.layers)
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reps} forwards of one {wl.name} layer (T={wl.T}, routed experts packed by the oracle), "
+                      f"{per_layer * 1e3:.1f} ms each, scaled to {wl.layers} layers per token"}
+
+
+def run_reference(args, wl: mi.Workload, rank: int, world: int):
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle_threads(wl)
+    steps_total = args.warmup + args.steps
+    logits_all = [[mi.router_logits(wl, l, s) for l in range(wl.layers)] for s in range(steps_total)]
+    needed = set()
+    for s in range(steps_total):
+        for l in range(wl.layers):
+            needed |= set(oracle.route(logits_all[s][l], wl.k)[0].ravel().tolist())
+    layer = OracleLayer(wl, 0, sorted(needed))
+    x = mi.activations(wl, 0, 0)
+    # size each step so that the whole run stays near two minutes: a step runs `per_step` of
+    # the workload's layers and counts as per_step / layers of a token
+    t0 = time.perf_counter()
+    layer.forward(x, logits_all[0][0], threads)
+    t_layer = time.perf_counter() - t0
+    per_step = int(max(1, min(wl.layers, round(120.0 / steps_total / max(t_layer, 1e-6)))))
+    for s in range(args.warmup):
+        for l in range(per_step):
+            layer.forward(x, logits_all[s][l], threads)
+    t0 = time.perf_counter()
+    for s in range(args.warmup, steps_total):
+        for l in range(per_step):
+            layer.forward(x, logits_all[s][l], threads)
+    el = time.perf_counter() - t0
+    value = wl.T * args.steps * per_step / wl.layers / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": config_of(wl, args, "oracle"),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"every step = {per_step} of the {wl.layers} layer forwards of a token "
+                                       f"(one {wl.name} layer's packed bank, T={wl.T}, fresh logits per layer "
+                                       f"and step) on the host cores"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(wl: mi.Workload, args, path: str):
+    return {"workload": wl.name, "layers": wl.layers, "hidden": wl.H, "intermediate": wl.I, "experts": wl.E,
+            "top_k": wl.k, "tokens_per_step": wl.T, "slots": wl.slots or wl.E, "routing": wl.routing,
+            "path": path, "l2": "inputs larger than L2 (packed bank of all layers, fresh routing per step)"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+class DecodeBench:
+    """All layers resident; per-step inputs resident; one CUDA graph per distinct step."""
+
+    RING = 32   # distinct step inputs (fresh routing each); replayed cyclically
+
+    def __init__(self, wl: mi.Workload, path: str, device):
+        import quantized_mixture_experts_grouped_b200 as q
+        self.q, self.wl, self.dev = q, wl, device
+        self.flags = q.PATHS[path]
+        H, I, E, k, T, Ls = wl.H, wl.I, wl.E, wl.k, wl.T, wl.layers
+        self.banks = []
+        for l in range(Ls):
+            w13b, w2b = mi.device_bank_weights(wl, l, device)
+            w13, s13 = q.alloc_bank(E, 2 * I, H, device)
+            w2, s2 = q.alloc_bank(E, H, I, device)
+            q.moe_quantize_pack(w13b, w13, s13)
+            q.moe_quantize_pack(w2b, w2, s2)
+            del w13b, w2b
+            self.banks.append((w13, s13, w2, s2))
+        torch.cuda.synchronize()
+        R = self.RING
+        # per ring slot, per layer: x [T][H] and logits [T][E], one contiguous block per slot
+        self.in_elems = Ls * (T * H + T * E)
+        host = np.empty((R, self.in_elems), np.uint16)
+        for r in range(R):
+            parts = []
+            for l in range(Ls):
+                parts.append(mi.activations(wl, l, r).ravel())
+                parts.append(mi.router_logits(wl, l, r).ravel())
+            host[r] = np.concatenate(parts)
+        self.inputs_host = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.inputs = self.inputs_host.to(device)
+        self.staging = torch.empty(self.in_elems, dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((R, Ls, T, H), dtype=torch.bfloat16, device=device)
+        self.out_e2e = torch.empty((Ls, T, H), dtype=torch.bfloat16, device=device)
+        self.out_host = torch.empty((Ls, T, H), dtype=torch.bfloat16).pin_memory()
+        self.idx = torch.empty((Ls, T, k), dtype=torch.int32, device=device)
+        self.wts = torch.empty((Ls, T, k), dtype=torch.float32, device=device)
+        self.ws = q.alloc_workspace(T, H, I, E, k, device)
+        self.stream = torch.cuda.Stream(device)
+
+    def _views(self, buf, l):
+        wl = self.wl
+        off = l * (wl.T * wl.H + wl.T * wl.E)
+        x = buf[off: off + wl.T * wl.H].view(wl.T, wl.H)
+        lg = buf[off + wl.T * wl.H: off + wl.T * wl.H + wl.T * wl.E].view(wl.T, wl.E)
+        return x, lg
+
+    def _layers(self, buf, out, events=None):
+        q, wl = self.q, self.wl
+        for l in range(wl.layers):
+            x, lg = self._views(buf, l)
+            w13, s13, w2, s2 = self.banks[l]
+            if events is not None:
+                events[2 * l].record(self.stream)
+            q.moe_w4a16_layer(x, lg, wl.k, w13, s13, w2, s2, wl.H, wl.I, self.idx[l], self.wts[l], self.ws,
+                              out[l], flags=self.flags, stream=self.stream)
+            if events is not None:
+                events[2 * l + 1].record(self.stream)
+
+    def capture(self):
+        q = self.q
+        self.graphs = []
+        torch.cuda.synchronize()
+        with torch.cuda.stream(self.stream):
+            self._layers(self.inputs[0], self.out[0])          # warm: lazy init outside capture
+        self.stream.synchronize()
+        n0 = q.moe_launch_count()
+        for r in range(self.RING):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self._layers(self.inputs[r], self.out[r])
+            self.graphs.append(g)
+        self.launches_per_step = (q.moe_launch_count() - n0) // self.RING
+        # the same steps with an event pair around every layer (kernel timing pass)
+        self.ev = []
+        self.ev_graphs = []
+        for r in range(self.RING):
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2 * self.wl.layers)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=self.stream):
+                self._layers(self.inputs[r], self.out[r], evs)
+            self.ev.append(evs)
+            self.ev_graphs.append(g)
+        # end-to-end: the layers read the step's inputs from a staging buffer that each step
+        # fills from pinned host memory; every layer's output goes back to pinned host memory
+        self.e2e_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.e2e_graph, stream=self.stream):
+            self._layers(self.staging, self.out_e2e)
+        torch.cuda.synchronize()
+
+    def e2e_step(self, r):
+        self.staging.copy_(self.inputs_host[r % self.RING], non_blocking=True)
+        self.e2e_graph.replay()
+        self.out_host.copy_(self.out_e2e, non_blocking=True)
+        self.stream.synchronize()           # the host reads the step's result
+
+    def run(self, graphs, n, start=0):
+        for i in range(n):
+            graphs[(start + i) % self.RING].replay()
+
+    def h2d_bytes(self):
+        return self.in_elems * 2
+
+    def d2h_bytes(self):
+        return self.out_e2e.numel() * 2
+
+
+def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
+    device = torch.device("cuda", local)
+    bench = DecodeBench(wl, args.path, device)
+    bench.capture()
+    s = bench.stream
+    peaks, peaks_kind = load_peaks()
+    sampler = ClockSampler(local)
+    with torch.cuda.stream(s):
+        bench.run(bench.graphs, args.warmup)
+        s.synchronize()
+        sampler.start()
+        # keep the GPU busy ~1.5 s so the clock sampler sees the regime the timed steps run in
+        t0 = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t0 < 1.5:
+            bench.run(bench.graphs, 64, i)
+            s.synchronize()
+            i += 64
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        bench.run(bench.graphs, args.steps, args.warmup)
+        e1.record(s)
+        e1.synchronize()
+        torch.cuda.synchronize()
+        barrier(world)
+        clocks = sampler.stop()
+        ms_total = all_max(e0.elapsed_time(e1), world)
+
+        # kernel timing pass: per-layer event pairs (one launch of the fused kernel per layer)
+        bench.run(bench.ev_graphs, max(3, args.warmup))
+        s.synchronize()
+        nk = max(args.steps, bench.RING)
+        durs = []
+        for i in range(nk):
+            r = i % bench.RING
+            bench.ev_graphs[r].replay()
+            s.synchronize()
+            evs = bench.ev[r]
+            durs.extend(evs[2 * l].elapsed_time(evs[2 * l + 1]) for l in range(wl.layers))
+        layer_ms = statistics.fmean(durs)
+
+        # end to end through host buffers
+        for i in range(max(3, args.warmup)):
+            bench.e2e_step(i)
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s)
+        for i in range(args.steps):
+            bench.e2e_step(args.warmup + i)
+        f1.record(s)
+        f1.synchronize()
+        e2e_ms = all_max(f0.elapsed_time(f1), world)
+    status = bench.q.moe_workspace_status(bench.ws, s)
+
+    if rank != 0:
+        return
+    tokens = wl.T * args.steps * world
+    value = tokens / (ms_total / 1e3)
+    bytes_per_layer = 8 * expert_bytes(wl.H, wl.I) if wl.T == 1 else None
+    achieved = bytes_per_layer / (layer_ms / 1e3) / 1e9
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(wl, args, args.path), us_per_layer=ms_total / args.steps / wl.layers * 1e3),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None,
+                     "kernel": "one moe_w4a16_layer launch sequence per layer (event pair per layer)",
+                     "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,
+                     "peak_kind": f"{peaks_kind} HBM copy"},
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d_bytes(),
+                "d2h_bytes_per_step": bench.d2h_bytes()},
+        "gpu_launches": bench.launches_per_step * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="olmoe_decode", choices=["olmoe_decode"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    wl = mi.WORKLOADS[args.workload]
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, wl, rank, world)
+        else:
+            run_ours(args, wl, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+// GPU-resident expert slot cache refilled from pinned host memory ("Every Expert Counts:
+// ExactMoE for Memory-Efficient W4A16 Inference", Abstract: experts stored in pinned host
+// memory and executed through a configurable GPU-resident slot cache).
+//
+// Host-side LRU bookkeeping; refills are cudaMemcpyAsync copies on a caller-given copy stream,
+// ordered after the last kernel that read the pool through an event. A routed set larger than
+// the pool runs in waves; the FFN of each wave sees only that wave's experts (others -1) and
+// accumulates into the workspace's fp32 accumulator, the last wave writing the bf16 output.
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "common.cuh"
+
+struct moe_slot_cache {
+  int E, S, H, I;
+  const uint8_t* bank_w13; const uint16_t* bank_s13;
+  const uint8_t* bank_w2; const uint16_t* bank_s2;
+  uint8_t* pool_w13; uint16_t* pool_s13;
+  uint8_t* pool_w2; uint16_t* pool_s2;
+  size_t w13_bytes, s13_bytes, w2_bytes, s2_bytes;   // per expert
+  std::vector<int32_t> slot_expert;                  // [S], -1 free
+  std::vector<int64_t> last_used;                    // [S]
+  int64_t clock = 0;
+  cudaEvent_t compute_done = nullptr;                // last FFN that read the pool
+  cudaEvent_t loaded = nullptr;
+  std::vector<int32_t> wave_tables;                  // host copies of every wave's table
+  std::vector<int32_t> idx_host;
+  int fail_copies_after = -1;                        // test hook: fail the n-th next copy
+};
+
+namespace moe {
+
+// Test hook: makes the n-th next refill copy (0 = the next one) of this cache report failure
+// as if cudaMemcpyAsync had returned an error; -1 disables.
+MOE_API void moe_slot_cache_fail_copy_after(moe_slot_cache* c, int n) {
+  if (c) c->fail_copies_after = n;
+}
+
+namespace {
+
+cudaError_t refill_copy(moe_slot_cache* c, void* dst, const void* src, size_t bytes, cudaStream_t s) {
+  if (c->fail_copies_after == 0) {
+    c->fail_copies_after = -1;
+    return cudaErrorInvalidValue;
+  }
+  if (c->fail_copies_after > 0) c->fail_copies_after--;
+  return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+MOE_API int moe_slot_cache_create(int E, int S, int H, int I, const uint8_t* bank_w13, const uint16_t* bank_s13,
+                                  const uint8_t* bank_w2, const uint16_t* bank_s2, uint8_t* pool_w13,
+                                  uint16_t* pool_s13, uint8_t* pool_w2, uint16_t* pool_s2, moe_slot_cache** out) {
+  if (!out) return fail(MOE_ERR_ARG, "moe_slot_cache_create: null out");
+  *out = nullptr;
+  if (E < 1 || S < 1 || E > kMaxExperts) return fail(MOE_ERR_ARG, "moe_slot_cache_create: E=%d S=%d", E, S);
+  if (H <= 0 || I <= 0 || H % kRowBlock || I % kRowBlock)
+    return fail(MOE_ERR_SHAPE, "moe_slot_cache_create: H=%d I=%d must be multiples of 128", H, I);
+  if (!bank_w13 || !bank_s13 || !bank_w2 || !bank_s2 || !pool_w13 || !pool_s13 || !pool_w2 || !pool_s2)
+    return fail(MOE_ERR_ARG, "moe_slot_cache_create: null bank or pool pointer");
+  moe_slot_cache* c = new moe_slot_cache();
+  c->E = E; c->S = S; c->H = H; c->I = I;
+  c->bank_w13 = bank_w13; c->bank_s13 = bank_s13; c->bank_w2 = bank_w2; c->bank_s2 = bank_s2;
+  c->pool_w13 = pool_w13; c->pool_s13 = pool_s13; c->pool_w2 = pool_w2; c->pool_s2 = pool_s2;
+  c->w13_bytes = (size_t)2 * I * H / 2;
+  c->s13_bytes = sizeof(uint16_t) * (size_t)2 * I * (H / kGroup);
+  c->w2_bytes = (size_t)H * I / 2;
+  c->s2_bytes = sizeof(uint16_t) * (size_t)H * (I / kGroup);
+  c->slot_expert.assign(S, -1);
+  c->last_used.assign(S, 0);
+  c->wave_tables.assign((size_t)E * (E + 1), -1);
+  if (int rc = check_cuda(cudaEventCreateWithFlags(&c->compute_done, cudaEventDisableTiming), "event create")) {
+    delete c;
+    return rc;
+  }
+  if (int rc = check_cuda(cudaEventCreateWithFlags(&c->loaded, cudaEventDisableTiming), "event create")) {
+    cudaEventDestroy(c->compute_done);
+    delete c;
+    return rc;
+  }
+  *out = c;
+  return MOE_OK;
+}
+
+MOE_API void moe_slot_cache_destroy(moe_slot_cache* c) {
+  if (!c) return;
+  if (c->compute_done) cudaEventDestroy(c->compute_done);
+  if (c->loaded) cudaEventDestroy(c->loaded);
+  delete c;
+}
+
+MOE_API int64_t moe_slot_cache_state(const moe_slot_cache* c, int32_t* slot_expert, int64_t* last_used) {
+  if (!c) return -1;
+  if (slot_expert) std::copy(c->slot_expert.begin(), c->slot_expert.end(), slot_expert);
+  if (last_used) std::copy(c->last_used.begin(), c->last_used.end(), last_used);
+  return c->clock;
+}
+
+MOE_API int slot_table_update(moe_slot_cache* c, uint64_t* needed_mask, int32_t* wave_table, int32_t* misses,
+                              int* n_misses, moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded) {
+  if (!c || !needed_mask || !wave_table || !misses || !n_misses)
+    return fail(MOE_ERR_ARG, "slot_table_update: null pointer");
+  const int E = c->E, S = c->S;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+  auto needed = [&](int e) { return (needed_mask[e >> 6] >> (e & 63)) & 1ull; };
+  std::vector<int> slot_of(E, -1);
+  for (int s = 0; s < S; ++s)
+    if (c->slot_expert[s] >= 0) slot_of[c->slot_expert[s]] = s;
+  std::vector<int> hits, miss;
+  for (int e = 0; e < E; ++e)
+    if (needed(e)) (slot_of[e] >= 0 ? hits : miss).push_back(e);
+  std::vector<char> in_wave(E, 0);
+  for (int e : hits) in_wave[e] = 1;
+  const int n_new = std::min(S - (int)hits.size(), (int)miss.size());
+  for (int i = 0; i < n_new; ++i) in_wave[miss[i]] = 1;
+
+  // plan on a copy of the state so that a failed copy can leave the committed state alone
+  std::vector<int32_t> se = c->slot_expert;
+  std::vector<int> loads_e, loads_s;
+  for (int i = 0; i < n_new; ++i) {
+    const int e = miss[i];
+    int pick = -1;
+    for (int s = 0; s < S && pick < 0; ++s)
+      if (se[s] < 0) pick = s;
+    if (pick < 0)
+      for (int s = 0; s < S; ++s) {
+        if (se[s] >= 0 && in_wave[se[s]]) continue;
+        if (pick < 0 || c->last_used[s] < c->last_used[pick]) pick = s;
+      }
+    if (pick < 0) return fail(MOE_ERR_ARG, "slot_table_update: no evictable slot (internal)");
+    if (se[pick] >= 0) slot_of[se[pick]] = -1;
+    se[pick] = e;
+    slot_of[e] = pick;
+    loads_e.push_back(e);
+    loads_s.push_back(pick);
+  }
+
+  if (!loads_e.empty() && reuse_ok)
+    if (int rc = check_cuda(cudaStreamWaitEvent(cs, reinterpret_cast<cudaEvent_t>(reuse_ok), 0),
+                            "slot_table_update: wait for pool reuse"))
+      return rc;
+  for (size_t i = 0; i < loads_e.size(); ++i) {
+    const size_t e = loads_e[i], s = loads_s[i];
+    cudaError_t err = refill_copy(c, c->pool_w13 + s * c->w13_bytes, c->bank_w13 + e * c->w13_bytes, c->w13_bytes, cs);
+    if (err == cudaSuccess)
+      err = refill_copy(c, reinterpret_cast<char*>(c->pool_s13) + s * c->s13_bytes,
+                        reinterpret_cast<const char*>(c->bank_s13) + e * c->s13_bytes, c->s13_bytes, cs);
+    if (err == cudaSuccess)
+      err = refill_copy(c, c->pool_w2 + s * c->w2_bytes, c->bank_w2 + e * c->w2_bytes, c->w2_bytes, cs);
+    if (err == cudaSuccess)
+      err = refill_copy(c, reinterpret_cast<char*>(c->pool_s2) + s * c->s2_bytes,
+                        reinterpret_cast<const char*>(c->bank_s2) + e * c->s2_bytes, c->s2_bytes, cs);
+    if (err != cudaSuccess) {
+      // slots written so far no longer hold what the committed state says: mark them free
+      for (size_t j = 0; j <= i; ++j) c->slot_expert[loads_s[j]] = -1;
+      *n_misses = 0;
+      return fail(MOE_ERR_CUDA, "slot_table_update: refill of expert %zu into slot %zu failed: %s", e, s,
+                  cudaGetErrorString(err));
+    }
+  }
+  if (loaded)
+    if (int rc = check_cuda(cudaEventRecord(reinterpret_cast<cudaEvent_t>(loaded), cs), "slot_table_update: record"))
+      return rc;
+
+  c->slot_expert = se;
+  for (int e = 0; e < E; ++e) {
+    wave_table[e] = in_wave[e] ? slot_of[e] : -1;
+    if (in_wave[e]) {
+      c->last_used[slot_of[e]] = c->clock;
+      needed_mask[e >> 6] &= ~(1ull << (e & 63));
+    }
+  }
+  c->clock += 1;
+  for (size_t i = 0; i < loads_e.size(); ++i) misses[i] = loads_e[i];
+  *n_misses = (int)loads_e.size();
+  return MOE_OK;
+}
+
+MOE_API int moe_slot_cache_layer(moe_slot_cache* c, const uint16_t* x, const uint16_t* logits, int T, int k,
+                                 int32_t* idx, float* wts, int32_t* wave_tables, void* workspace,
+                                 size_t workspace_bytes, uint16_t* out, int path, moe_stream_t stream,
+                                 moe_stream_t copy_stream, int* n_waves, int* n_loads) {
+  if (!c || !wave_tables || !n_waves || !n_loads) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: null pointer");
+  if (T < 0 || k < 1 || k > c->E) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: bad sizes");
+  *n_waves = 0;
+  *n_loads = 0;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int E = c->E;
+  if (int rc = moe_route_topk(logits, T, E, k, idx, wts, stream)) return rc;
+  c->idx_host.resize((size_t)T * k);
+  if (int rc = check_cuda(cudaMemcpyAsync(c->idx_host.data(), idx, sizeof(int32_t) * T * k, cudaMemcpyDeviceToHost, s),
+                          "moe_slot_cache_layer: read routed experts"))
+    return rc;
+  if (int rc = check_cuda(cudaStreamSynchronize(s), "moe_slot_cache_layer: sync")) return rc;
+  uint64_t mask[kMaxExperts / 64] = {0, 0, 0, 0};
+  for (int32_t e : c->idx_host) {
+    if (e < 0 || e >= E) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: routed expert %d out of range", e);
+    mask[e >> 6] |= 1ull << (e & 63);
+  }
+  std::vector<int32_t> miss(c->S);
+  int wave = 0;
+  auto any = [&]() { return (mask[0] | mask[1] | mask[2] | mask[3]) != 0; };
+  while (any()) {
+    if (wave > (E + c->S - 1) / c->S) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: too many waves (internal)");
+    int32_t* table_h = c->wave_tables.data() + (size_t)wave * E;
+    int nm = 0;
+    if (int rc = slot_table_update(c, mask, table_h, miss.data(), &nm, copy_stream,
+                                   reinterpret_cast<moe_event_t>(c->compute_done),
+                                   reinterpret_cast<moe_event_t>(c->loaded)))
+      return rc;
+    *n_loads += nm;
+    int32_t* table_d = wave_tables + (size_t)wave * E;
+    if (int rc = check_cuda(cudaMemcpyAsync(table_d, table_h, sizeof(int32_t) * E, cudaMemcpyHostToDevice, s),
+                            "moe_slot_cache_layer: upload wave table"))
+      return rc;
+    if (int rc = check_cuda(cudaStreamWaitEvent(s, c->loaded, 0), "moe_slot_cache_layer: wait refill")) return rc;
+    const bool last = !any();
+    const int flags = (path & MOE_PATH_MASK) | (wave > 0 ? MOE_FLAG_ACCUMULATE : 0);
+    if (int rc = moe_w4a16_ffn(x, T, c->H, c->I, E, k, idx, wts, c->pool_w13, c->pool_s13, c->pool_w2, c->pool_s2,
+                               table_d, workspace, workspace_bytes, last ? out : nullptr,
+                               last ? flags : (flags | MOE_FLAG_ACCUMULATE), stream))
+      return rc;
+    if (int rc = check_cuda(cudaEventRecord(c->compute_done, s), "moe_slot_cache_layer: record")) return rc;
+    ++wave;
+  }
+  *n_waves = wave;
+  return MOE_OK;
+}

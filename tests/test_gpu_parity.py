@@ -1,0 +1,340 @@
+"""GPU parity: every CUDA kernel, called through the C ABI, against the CPU oracle.
+
+Bit-exact: packed codes and scales, router indices, grouping (counts/offsets/perm/inv), slot
+tables. Floating point: router weights to ROUTE_RTOL; FFN outputs to max-abs 2e-2 and
+relative L2 5e-3 against the oracle on the same dequantised weights (the packed bytes the
+oracle produced are uploaded unchanged). Sizes span several tiles and ragged tails; the
+full-size workloads are checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+from gpu_util import (Layer, assert_ffn_close, bits_to_dev, dev_to_bits, bf16_dev_to_f32, ROUTE_RTOL)
+
+pytestmark = pytest.mark.gpu
+
+q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
+
+FFN_PATHS = ["simple"]
+
+
+def _ws(T, H, I, E, k):
+    return q.alloc_workspace(T, H, I, E, k)
+
+
+# ----------------------------------------------------------------------------- pack
+
+def _pack_on_gpu(w_bits: np.ndarray):
+    E, N, K = w_bits.shape
+    w = bits_to_dev(w_bits)
+    packed, scales = q.alloc_bank(E, N, K)
+    q.moe_quantize_pack(w, packed, scales)
+    torch.cuda.synchronize()
+    return packed.cpu().numpy(), dev_to_bits(scales)
+
+
+@pytest.mark.parametrize("dist", ["normal", "heavy_zero_groups", "ties"])
+def test_pack_bit_exact_small(dist):
+    g = np.random.default_rng(7)
+    E, N, K = 3, 384, 512
+    if dist == "normal":
+        w = g.standard_normal((E, N, K)) * 0.02
+    elif dist == "heavy_zero_groups":
+        w = g.standard_t(2, (E, N, K)) * np.exp(g.uniform(-30, 3, (E, N, 1)))
+        w[:, 5, 128:256] = 0.0
+        w[1, 130:140, :] = 0.0
+    else:   # quarter-integer multiples of a power of two: many w/s exactly on .5
+        w = g.integers(-28, 29, (E, N, K)) * 0.125
+        w[..., 0] = 3.5
+    wb = mi.to_bf16_bits(w.astype(np.float32))
+    packed, scales = _pack_on_gpu(wb)
+    for e in range(E):
+        ref_p, ref_s = oracle.pack(*oracle.quantize(wb[e]))
+        np.testing.assert_array_equal(packed[e], ref_p)
+        np.testing.assert_array_equal(scales[e], ref_s)
+
+
+def test_pack_bit_exact_full_size_experts():
+    """OLMoE gate/up (2048x2048) and down (2048x1024) of two experts, and the large-expert
+    gate/up (28672x4096) of one expert."""
+    wl = mi.WORKLOADS["olmoe_decode"]
+    for e in (0, 63):
+        a, b = mi.expert_weights(wl, 3, e)
+        for m in (a, b):
+            packed, scales = _pack_on_gpu(m[None])
+            ref_p, ref_s = oracle.pack(*oracle.quantize(m))
+            np.testing.assert_array_equal(packed[0], ref_p)
+            np.testing.assert_array_equal(scales[0], ref_s)
+    wl = mi.WORKLOADS["large_expert"]
+    a, _ = mi.expert_weights(wl, 0, 5)
+    packed, scales = _pack_on_gpu(a[None])
+    ref_p, ref_s = oracle.pack(*oracle.quantize(a))
+    np.testing.assert_array_equal(packed[0], ref_p)
+    np.testing.assert_array_equal(scales[0], ref_s)
+
+
+# ----------------------------------------------------------------------------- route
+
+def _route_gpu(lb: np.ndarray, k: int):
+    T, E = lb.shape
+    logits = bits_to_dev(lb)
+    idx = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    q.moe_route_topk(logits, k, idx, wts)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), wts.cpu().numpy()
+
+
+@pytest.mark.parametrize("T,E,k,kind", [(4, 8, 2, "normal"), (2048, 64, 8, "zipf"), (2048, 64, 8, "normal"),
+                                        (17, 64, 64, "ties"), (33, 256, 8, "ties"), (512, 8, 2, "normal"),
+                                        (5, 3, 1, "ties"), (1, 64, 8, "normal")])
+def test_route_matches_oracle(T, E, k, kind):
+    g = np.random.default_rng(T + E + k)
+    if kind == "zipf":
+        wl = mi.Workload("z", H=128, I=128, E=E, k=k, T=T, routing="zipf")
+        lb = mi.router_logits(wl, 0, 0)
+    else:
+        l = g.standard_normal((T, E)).astype(np.float32)
+        if kind == "ties":
+            l = np.round(l * 2) / 2
+            l[:, 1::5] = -0.0
+            l[:, 2::5] = 0.0
+        lb = mi.to_bf16_bits(l)
+    idx, wts = _route_gpu(lb, k)
+    ridx, rwts = oracle.route(lb, k)
+    np.testing.assert_array_equal(idx, ridx)
+    np.testing.assert_allclose(wts, rwts, rtol=ROUTE_RTOL, atol=0)
+
+
+def test_route_empty_batch_is_noop():
+    idx = torch.full((1, 2), -7, dtype=torch.int32, device="cuda")
+    wts = torch.zeros((1, 2), device="cuda")
+    q.lib.moe_route_topk(None, 0, 8, 2, None, None, None) == 0
+    assert (idx == -7).all()
+
+
+# ----------------------------------------------------------------------------- permute
+
+@pytest.mark.parametrize("T,E,k", [(1, 64, 8), (16, 64, 8), (2048, 64, 8), (3000, 256, 8), (4, 8, 2)])
+def test_permute_bit_exact(T, E, k):
+    g = np.random.default_rng(T * 7 + E)
+    if E == 64 and T == 2048:
+        wl = mi.Workload("z", H=128, I=128, E=E, k=k, T=T, routing="zipf")
+        idx, _ = oracle.route(mi.router_logits(wl), k)
+    else:
+        idx = np.stack([g.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    d_idx = torch.from_numpy(idx).cuda()
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    inv = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    scratch = torch.empty(max(1, q.moe_permute_scratch_count(T, k, E)), dtype=torch.int32, device="cuda")
+    q.moe_permute(d_idx, E, counts, offsets, perm, inv, scratch)
+    torch.cuda.synchronize()
+    rc, ro, rp, ri = oracle.permute(idx, E)
+    np.testing.assert_array_equal(counts.cpu().numpy(), rc)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), ro)
+    np.testing.assert_array_equal(perm.cpu().numpy(), rp)
+    np.testing.assert_array_equal(inv.cpu().numpy(), ri)
+
+
+# ----------------------------------------------------------------------------- FFN
+
+def _run_ffn(layer: Layer, path: str, out=None, slot=None):
+    d = layer.to_device()
+    wl = layer.wl
+    ws = _ws(layer.T, wl.H, wl.I, wl.E, wl.k)
+    out = torch.empty((layer.T, wl.H), dtype=torch.bfloat16, device="cuda") if out is None else out
+    q.moe_w4a16_ffn(d["x"], d["idx"], d["wts"], d["w13"], d["s13"], d["w2"], d["s2"], wl.H, wl.I, wl.E, ws, out,
+                    slot_of_expert=slot, flags=q.PATHS[path])
+    torch.cuda.synchronize()
+    assert q.moe_workspace_status(ws) == 0
+    return out, ws
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+@pytest.mark.parametrize("T", [4, 1, 17, 64])
+def test_ffn_tiny_shapes(path, T):
+    layer = Layer(mi.WORKLOADS["tiny"], T=T)
+    out, _ = _run_ffn(layer, path)
+    assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"tiny T={T} {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_edge_cases(path):
+    wl = mi.Workload("edge", H=384, I=256, E=8, k=3, T=37)
+    g = np.random.default_rng(2)
+    # one expert takes every token (its logit dominates), two experts get none
+    l = g.standard_normal((wl.T, wl.E)).astype(np.float32)
+    l[:, 5] += 100.0
+    l[:, 0] -= 100.0
+    l[:, 7] -= 100.0
+    layer = Layer(wl, logits=mi.to_bf16_bits(l))
+    # an all-zero weight group in one expert
+    layer.w13[5][:8192] = 0x88      # code 8 = q 0 for a whole tile
+    out, _ = _run_ffn(layer, path)
+    assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge {path}")
+    # k = E: every expert on every token
+    wl2 = mi.Workload("kE", H=256, I=128, E=4, k=4, T=9)
+    layer2 = Layer(wl2)
+    out2, _ = _run_ffn(layer2, path)
+    assert_ffn_close(bf16_dev_to_f32(out2), layer2.oracle_out(), f"k=E {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_olmoe_decode_and_batched(path):
+    for name, T in (("olmoe_decode", 1), ("olmoe_slots", 16)):
+        wl = mi.WORKLOADS[name]
+        probe = Layer(mi.Workload("p", H=128, I=128, E=wl.E, k=wl.k, T=T, routing=wl.routing, seed=wl.seed),
+                      layer=2, step=5, experts=[])
+        routed = sorted(set(probe.idx.ravel().tolist()))
+        layer = Layer(wl, layer=2, step=5, T=T, experts=routed, logits=probe.logits)
+        out, _ = _run_ffn(layer, path)
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"{name} {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_prefill_full_size_sampled(path):
+    wl = mi.WORKLOADS["olmoe_prefill"]
+    layer = Layer(wl)
+    counts = np.bincount(layer.idx.ravel(), minlength=wl.E)
+    assert counts.max() > 1000 and counts.min() < 200      # Zipf skew reached the kernels
+    out, _ = _run_ffn(layer, path)
+    got = bf16_dev_to_f32(out)
+    assert np.all(np.isfinite(got))
+    tokens = [0, 1, 777, 1024, 2047]
+    assert_ffn_close(got[tokens], layer.oracle_out(tokens=tokens), f"prefill {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_large_expert_full_size_sampled(path):
+    wl = mi.WORKLOADS["large_expert"]
+    layer = Layer(wl)
+    out, _ = _run_ffn(layer, path)
+    got = bf16_dev_to_f32(out)
+    assert np.all(np.isfinite(got))
+    tokens = [0, 255, 511]
+    assert_ffn_close(got[tokens], layer.oracle_out(tokens=tokens), f"large {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_deterministic_and_slot_indirection(path):
+    layer = Layer(mi.WORKLOADS["tiny"], T=19)
+    a, _ = _run_ffn(layer, path)
+    b, _ = _run_ffn(layer, path)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    # the same experts stored in permuted slots through the expert -> slot table
+    d = layer.to_device()
+    E = layer.wl.E
+    perm = np.random.default_rng(0).permutation(E).astype(np.int32)     # expert e lives in slot perm[e]
+    w13 = torch.empty_like(d["w13"]); s13 = torch.empty_like(d["s13"])
+    w2 = torch.empty_like(d["w2"]); s2 = torch.empty_like(d["s2"])
+    for e in range(E):
+        w13[perm[e]] = d["w13"][e]; s13[perm[e]] = d["s13"][e]
+        w2[perm[e]] = d["w2"][e]; s2[perm[e]] = d["s2"][e]
+    table = torch.from_numpy(perm).cuda()
+    ws = _ws(layer.T, layer.wl.H, layer.wl.I, E, layer.wl.k)
+    c = torch.empty_like(a)
+    q.moe_w4a16_ffn(d["x"], d["idx"], d["wts"], w13, s13, w2, s2, layer.wl.H, layer.wl.I, E, ws, c,
+                    slot_of_expert=table, flags=q.PATHS[path])
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_wave_accumulation(path):
+    """Experts split into two waves (slot -1 skips), accumulated in fp32, equal one pass."""
+    layer = Layer(mi.WORKLOADS["tiny"], T=11)
+    d = layer.to_device()
+    wl = layer.wl
+    ws = _ws(layer.T, wl.H, wl.I, wl.E, wl.k)
+    t1 = torch.tensor([e if e < 4 else -1 for e in range(wl.E)], dtype=torch.int32, device="cuda")
+    t2 = torch.tensor([e if e >= 4 else -1 for e in range(wl.E)], dtype=torch.int32, device="cuda")
+    out = torch.empty((layer.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    args = (d["x"], d["idx"], d["wts"], d["w13"], d["s13"], d["w2"], d["s2"], wl.H, wl.I, wl.E, ws)
+    q.moe_w4a16_ffn(*args, None, slot_of_expert=t1, flags=q.PATHS[path] | q.MOE_FLAG_ACCUMULATE)
+    q.moe_w4a16_ffn(*args, out, slot_of_expert=t2, flags=q.PATHS[path] | q.MOE_FLAG_ACCUMULATE)
+    torch.cuda.synchronize()
+    assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"waves {path}")
+    # the accumulator was cleared again: a plain call gives the same answer
+    out2, _ = _run_ffn(layer, path)
+    assert_ffn_close(bf16_dev_to_f32(out2), layer.oracle_out(), f"after waves {path}")
+
+
+# ----------------------------------------------------------------------------- slot cache
+
+def _make_cache(wl: mi.Workload, S: int, layer: Layer):
+    E = wl.E
+    bank = [torch.from_numpy(layer.w13).pin_memory(),
+            torch.from_numpy(layer.s13.view(np.int16)).view(torch.bfloat16).pin_memory(),
+            torch.from_numpy(layer.w2).pin_memory(),
+            torch.from_numpy(layer.s2.view(np.int16)).view(torch.bfloat16).pin_memory()]
+    pool = [torch.zeros((S,) + tuple(b.shape[1:]), dtype=b.dtype, device="cuda") for b in bank]
+    return q.SlotCache(E, S, wl.H, wl.I, bank, pool)
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_slot_cache_layer_matches_oracle(path):
+    wl = mi.Workload("cache", H=256, I=128, E=8, k=3, T=3)
+    base = Layer(wl)
+    S = 3
+    cache = _make_cache(wl, S, base)
+    ref_state = oracle.SlotState(wl.E, S)
+    copy_stream = torch.cuda.Stream()
+    ws = _ws(wl.T, wl.H, wl.I, wl.E, wl.k)
+    wave_tables = torch.empty(wl.E * (wl.E // S + 2), dtype=torch.int32, device="cuda")
+    total_waves = 0
+    for step in range(12):
+        layer = Layer(wl, step=step, experts=[])
+        layer.w13, layer.s13, layer.w2, layer.s2 = base.w13, base.s13, base.w2, base.s2
+        d = layer.to_device()
+        idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+        out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+        n_waves, n_loads = cache.layer(d["x"], d["logits"], wl.k, idx, wts, wave_tables, ws, out, path=q.PATHS[path],
+                                       copy_stream=copy_stream)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
+        # replay the oracle's LRU policy wave by wave
+        needed = np.zeros(wl.E, np.uint8)
+        needed[np.unique(layer.idx)] = 1
+        waves = loads = 0
+        while needed.any():
+            _, ld = ref_state.wave(needed)
+            waves += 1
+            loads += len(ld)
+        assert (n_waves, n_loads) == (waves, loads)
+        se, lu, clock = cache.state()
+        np.testing.assert_array_equal(se, ref_state.slot_expert)
+        np.testing.assert_array_equal(lu, ref_state.last_used)
+        assert clock == ref_state.clock[0]
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"cache step {step}")
+        total_waves += n_waves
+    assert total_waves > 12          # some steps needed more than one wave (k*T > S)
+
+
+def test_slot_table_update_refill_failure_is_reported():
+    wl = mi.Workload("cachefail", H=256, I=128, E=8, k=2, T=2)
+    base = Layer(wl, experts=range(8))
+    cache = _make_cache(wl, 2, base)
+    copy_stream = torch.cuda.Stream()
+    mask = np.array([0b00000110], dtype=np.uint64)         # experts 1 and 2
+    table = np.zeros(wl.E, np.int32)
+    misses = np.zeros(2, np.int32)
+    cache.fail_copy_after(5)      # expert 1's four copies succeed, expert 2's second copy fails
+    with pytest.raises(q.MoeError) as ei:
+        cache.slot_table_update(mask, table, misses, copy_stream)
+    assert ei.value.code == q.MOE_ERR_CUDA
+    se, _, clock = cache.state()
+    assert se.tolist() == [-1, -1] and clock == 0 and mask[0] == 0b110     # nothing committed
+    # the next attempt succeeds and loads both
+    n = cache.slot_table_update(mask, table, misses, copy_stream)
+    torch.cuda.synchronize()
+    assert n == 2 and misses.tolist() == [1, 2] and mask[0] == 0
+    assert table.tolist() == [-1, 0, 1, -1, -1, -1, -1, -1]
+    pool_w13 = cache.pool[0].cpu().numpy()
+    np.testing.assert_array_equal(pool_w13[0], base.w13[1])
+    np.testing.assert_array_equal(pool_w13[1], base.w13[2])
