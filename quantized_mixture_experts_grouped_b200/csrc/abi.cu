@@ -51,7 +51,7 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
   L.hp = take(sizeof(uint16_t) * Tk * I);
   L.yp = take(sizeof(float) * Tk * H);
   L.acc = take(sizeof(float) * (size_t)T * H);
-  L.dec = take(0);
+  L.dec = take(decode_scratch_bytes(T, H, I, E, k));
   L.total = off;
   return L;
 }
@@ -83,6 +83,8 @@ int check_layer_args(const uint16_t* x, int T, int H, int I, int E, int k, const
     return fail(MOE_ERR_ARG, "x and out must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(w13) | reinterpret_cast<uintptr_t>(w2)) & 127)
     return fail(MOE_ERR_ARG, "packed weights must be 128-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(s13) | reinterpret_cast<uintptr_t>(s2)) & 15)
+    return fail(MOE_ERR_ARG, "scales must be 16-byte aligned");
   return MOE_OK;
 }
 

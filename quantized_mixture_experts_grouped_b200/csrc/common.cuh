@@ -58,6 +58,7 @@ enum CtlWord {
 };
 
 size_t permute_scratch_count(int T, int k, int E);
+size_t decode_scratch_bytes(int T, int H, int I, int E, int k);
 
 // ---- launch helpers (defined in the .cu files) ----
 int launch_quantize_pack(const uint16_t* w, int E, int N, int K, uint8_t* packed, uint16_t* scales,

@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(128) route_kernel(const uint16_t* __restrict__
       lv[i] = -INFINITY;
     }
   }
-  int chosen_e = -1;     // lane j (< k) keeps the j-th choice
+  int chosen[kMaxPerLane];   // lane (j % 32) keeps choice j in chosen[j / 32]
   float mx = 0.f;
   for (int j = 0; j < k; ++j) {
     uint32_t best = 0;
@@ -55,7 +55,9 @@ __global__ void __launch_bounds__(128) route_kernel(const uint16_t* __restrict__
     const uint32_t win = __reduce_max_sync(0xffffffffu, best);
     const int e = 0xffff - (int)(win & 0xffffu);
     if ((e & 31) == lane) taken |= 1u << (e >> 5);
-    if (lane == j) chosen_e = e;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i)
+      if (j == 32 * i + lane) chosen[i] = e;
     if (j == 0) {   // the largest logit, decoded back from its key
       const uint32_t ord = win >> 16;
       mx = bf16_bits_to_float((ord & 0x8000u) ? (ord & 0x7fffu) : (~ord & 0xffffu));
@@ -67,14 +69,23 @@ __global__ void __launch_bounds__(128) route_kernel(const uint16_t* __restrict__
     if (lane + 32 * i < E) z += expf(lv[i] - mx);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  float p = 0.f;
-  if (lane < k) p = expf(bf16_bits_to_float(lt[chosen_e]) - mx) / z;
-  float sel = p;
+  float p[kMaxPerLane];
+  float sel = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    p[i] = 0.f;
+    if (32 * i + lane < k) p[i] = expf(bf16_bits_to_float(lt[chosen[i]]) - mx) / z;
+    sel += p[i];
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sel += __shfl_xor_sync(0xffffffffu, sel, o);
-  if (lane < k) {
-    idx[(size_t)t * k + lane] = chosen_e;
-    wts[(size_t)t * k + lane] = p / sel;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int j = 32 * i + lane;
+    if (j < k) {
+      idx[(size_t)t * k + j] = chosen[i];
+      wts[(size_t)t * k + j] = p[i] / sel;
+    }
   }
 }
 

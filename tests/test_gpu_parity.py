@@ -18,7 +18,13 @@ pytestmark = pytest.mark.gpu
 
 q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
 
-FFN_PATHS = ["simple"]
+FFN_PATHS = ["simple", "decode"]
+
+
+def _supported(path, T, k):
+    """The fused decode path takes small batches only (T <= 32 and T*k <= 256)."""
+    if path == "decode" and not (1 <= T <= 32 and T * k <= 256):
+        pytest.skip("fused decode path is for small batches")
 
 
 def _ws(T, H, I, E, k):
@@ -112,7 +118,7 @@ def test_route_matches_oracle(T, E, k, kind):
 def test_route_empty_batch_is_noop():
     idx = torch.full((1, 2), -7, dtype=torch.int32, device="cuda")
     wts = torch.zeros((1, 2), device="cuda")
-    q.lib.moe_route_topk(None, 0, 8, 2, None, None, None) == 0
+    assert q.lib.moe_route_topk(None, 0, 8, 2, None, None, None) == 0
     assert (idx == -7).all()
 
 
@@ -144,6 +150,7 @@ def test_permute_bit_exact(T, E, k):
 # ----------------------------------------------------------------------------- FFN
 
 def _run_ffn(layer: Layer, path: str, out=None, slot=None):
+    _supported(path, layer.T, layer.wl.k)
     d = layer.to_device()
     wl = layer.wl
     ws = _ws(layer.T, wl.H, wl.I, wl.E, wl.k)
@@ -177,11 +184,52 @@ def test_ffn_edge_cases(path):
     layer.w13[5][:8192] = 0x88      # code 8 = q 0 for a whole tile
     out, _ = _run_ffn(layer, path)
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge {path}")
-    # k = E: every expert on every token
+
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_k_equals_e(path):
+    """k = E: every expert on every token."""
     wl2 = mi.Workload("kE", H=256, I=128, E=4, k=4, T=9)
     layer2 = Layer(wl2)
     out2, _ = _run_ffn(layer2, path)
     assert_ffn_close(bf16_dev_to_f32(out2), layer2.oracle_out(), f"k=E {path}")
+
+
+@pytest.mark.parametrize("path", FFN_PATHS)
+def test_ffn_edge_cases_small_batch(path):
+    """Decode-sized batch: one expert takes every token, two get none, one all-zero group."""
+    wl = mi.Workload("edge_small", H=384, I=256, E=8, k=3, T=21)
+    g = np.random.default_rng(3)
+    l = g.standard_normal((wl.T, wl.E)).astype(np.float32)
+    l[:, 2] += 100.0
+    l[:, 0] -= 100.0
+    l[:, 7] -= 100.0
+    layer = Layer(wl, logits=mi.to_bf16_bits(l))
+    layer.w2[2][8192:16384] = 0x88
+    out, _ = _run_ffn(layer, path)
+    assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
+
+
+@pytest.mark.parametrize("path", ["auto", "decode", "simple"])
+@pytest.mark.parametrize("T", [1, 5, 16])
+def test_layer_call_routes_and_runs(path, T):
+    """moe_w4a16_layer: routing (in-kernel on the fused path) + FFN in one call."""
+    wl = mi.Workload("layer", H=512, I=256, E=16, k=4, T=T)
+    layer = Layer(wl, layer=1, step=T)
+    d = layer.to_device()
+    ws = _ws(T, wl.H, wl.I, wl.E, wl.k)
+    idx = torch.full((T, wl.k), -1, dtype=torch.int32, device="cuda")
+    wts = torch.zeros((T, wl.k), dtype=torch.float32, device="cuda")
+    out = torch.empty((T, wl.H), dtype=torch.bfloat16, device="cuda")
+    for rep in range(2):
+        q.moe_w4a16_layer(d["x"], d["logits"], wl.k, d["w13"], d["s13"], d["w2"], d["s2"], wl.H, wl.I, idx, wts,
+                          ws, out, flags=q.PATHS[path])
+        torch.cuda.synchronize()
+        assert q.moe_workspace_status(ws) == 0
+        np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
+        np.testing.assert_allclose(wts.cpu().numpy(), layer.wts, rtol=ROUTE_RTOL)
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"layer {path} T={T} rep={rep}")
 
 
 @pytest.mark.parametrize("path", FFN_PATHS)
@@ -223,6 +271,7 @@ def test_ffn_large_expert_full_size_sampled(path):
 @pytest.mark.parametrize("path", FFN_PATHS)
 def test_ffn_deterministic_and_slot_indirection(path):
     layer = Layer(mi.WORKLOADS["tiny"], T=19)
+    _supported(path, layer.T, layer.wl.k)
     a, _ = _run_ffn(layer, path)
     b, _ = _run_ffn(layer, path)
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
@@ -248,6 +297,7 @@ def test_ffn_deterministic_and_slot_indirection(path):
 def test_ffn_wave_accumulation(path):
     """Experts split into two waves (slot -1 skips), accumulated in fp32, equal one pass."""
     layer = Layer(mi.WORKLOADS["tiny"], T=11)
+    _supported(path, layer.T, layer.wl.k)
     d = layer.to_device()
     wl = layer.wl
     ws = _ws(layer.T, wl.H, wl.I, wl.E, wl.k)
