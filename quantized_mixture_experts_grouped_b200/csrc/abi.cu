@@ -2,6 +2,7 @@
 // dispatch to the kernel paths. Nothing here allocates device memory.
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <atomic>
 #include <string>
 
@@ -47,6 +48,12 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
   L.inv = take(sizeof(int32_t) * Tk);
   L.perm_scratch = take(sizeof(int32_t) * permute_scratch_count(T, k, E));
   L.tiles = take(sizeof(int32_t) * (4 * (E + 1) + 64));
+  {
+    const size_t chunks = (Tk + 127) / 128 + (size_t)E;
+    const size_t blocks = std::max<size_t>(I / 128, H / 256 + 1);
+    L.tile_list_len = chunks * blocks;
+    L.tile_list = take(sizeof(int32_t) * 2 * L.tile_list_len);
+  }
   L.xp = take(sizeof(uint16_t) * Tk * H);
   L.hp = take(sizeof(uint16_t) * Tk * I);
   L.yp = take(sizeof(float) * Tk * H);

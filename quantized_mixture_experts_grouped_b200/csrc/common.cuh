@@ -38,6 +38,8 @@ struct WsLayout {
   size_t inv;           // int32 [T*k]
   size_t perm_scratch;  // int32 permute scratch
   size_t tiles;         // int32 [E+1] tile prefix + misc
+  size_t tile_list;     // int32 [2][tile_list_len] grouped-GEMM tile lists (gate/up, down)
+  size_t tile_list_len;
   size_t xp;            // bf16 [T*k][H] gathered activations
   size_t hp;            // bf16 [T*k][I] SwiGLU intermediate
   size_t yp;            // fp32 [T*k][H] per-pair down projection (weighted in combine)

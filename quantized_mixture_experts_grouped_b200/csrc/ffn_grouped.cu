@@ -1,0 +1,572 @@
+// Grouped W4A16 GEMM path of the MoE layer for large token batches (prefill) ("Every Expert
+// Counts: ExactMoE for Memory-Efficient W4A16 Inference", Abstract: all selected experts run
+// through fused grouped MoE kernels).
+//
+// Launch sequence: permute (group pairs by expert) -> gather rows -> tile plan -> gate/up GEMM
+// with fused silu(g)*u -> down GEMM with the router weight fused in its epilogue -> combine.
+//
+// Both GEMMs are one persistent tcgen05 kernel (sm_100a). A CTA tile is a PAIR of 128-row
+// weight blocks (gate rows f..f+127 and the matching up rows, or two consecutive row blocks of
+// W2) against up to 128 tokens of one expert:
+//   D_0[128 x N] = W_blk0 . X^T,  D_1[128 x N] = W_blk1 . X^T   (N = tokens, multiple of 16)
+// The weights are the A operand and live in TENSOR MEMORY: 8 dequantiser warps turn each 128 x
+// 128 int4 tile (TMA-staged in shared memory) into bf16 rows (q * s) and write them with
+// tcgen05.st. The token rows are the B operand, loaded by TMA with 128-byte swizzle; one token
+// tile feeds both MMAs, which keeps the shared-memory traffic per MMA flop low. Accumulators
+// are fp32 in tensor memory; 4 epilogue warps drain them with tcgen05.ld.
+// Tile list: per expert, ceil(n_e / 128) token chunks x row-block pairs; MMA N is the chunk's
+// token count rounded up to 16, so a ragged tail costs at most 15 padded tokens per expert.
+// Tiles are claimed dynamically (atomic counter). Every wait is bounded.
+#include <algorithm>
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kGStages = 4;
+constexpr int kGThreads = 448;
+constexpr int kGEpi0 = 2;           // warps 2..5
+constexpr int kGDq0 = 6;            // warps 6..13
+constexpr int kTokTile = 128;
+constexpr int kGTmemCols = 512;
+constexpr int kGA = 0;              // 2 A buffers x (64 gate + 64 up) columns
+constexpr int kGD0 = 256;           // D_0 columns 256..383
+constexpr int kGD1 = 384;           // D_1 columns 384..511
+constexpr uint32_t kBBoxBytes = kTokTile * 128;   // one 64-wide K box of 128 rows (16 KB)
+
+enum { kModeGateUp = 0, kModeDown = 1 };
+
+struct __align__(1024) GStage {
+  uint8_t b[2][kBBoxBytes];     // token rows, K 0..63 and 64..127 of the group (SW128)
+  uint8_t w[2][8192];           // int4 tiles of block 0 and block 1
+  uint16_t sc[2][128];          // their scales
+};
+
+struct GSmem {
+  GStage st[kGStages];
+  uint64_t full[kGStages], empty[kGStages];
+  uint64_t afull[2], aempty[2];
+  uint64_t dfull, dempty;
+  uint64_t tq_full[4], tq_empty[4];
+  uint64_t drain;
+  int tq[4];
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct GParams {
+  const uint8_t* w; const uint16_t* s;     // packed bank of the matrix (per slot)
+  size_t w_stride, s_stride;                // per slot
+  int K;                                    // H for gate/up, I for down
+  int G;                                    // K / 128
+  int rows_half;                            // gate/up: I (up block offset); down: unused
+  int mode;
+  const int32_t* tile_list;                 // packed tiles
+  const int32_t* ntiles;                    // total tile count (device)
+  const int32_t* offsets;                   // grouped pair offsets [E+1]
+  const int32_t* table;                     // expert -> slot (nullable)
+  const int32_t* perm;                      // pair id of grouped position
+  const float* wts;                         // router weights [T*k]
+  uint16_t* out;                            // gate/up: Hp [Tk][I]; down: Yp [Tk][H] (weighted)
+  int out_ld;                               // row length of out
+  int Tk;
+  int* ctl;
+};
+
+// packed tile: expert (8 bits) | chunk (12 bits) | block pair (12 bits)
+__device__ __forceinline__ void unpack_tile(int32_t v, int& e, int& chunk, int& bp) {
+  e = (v >> 24) & 0xff;
+  chunk = (v >> 12) & 0xfff;
+  bp = v & 0xfff;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(tc::smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(tc::smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
+        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = tc::mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+struct TileDesc {
+  int e, slot, chunk, bp, p0, ntok;
+  size_t rb0, rb1;     // weight row blocks
+};
+
+__device__ __forceinline__ TileDesc describe(const GParams& P, int32_t packed) {
+  TileDesc d;
+  unpack_tile(packed, d.e, d.chunk, d.bp);
+  d.slot = slot_of(P.table, d.e);
+  const int n_e = P.offsets[d.e + 1] - P.offsets[d.e];
+  d.p0 = P.offsets[d.e] + d.chunk * kTokTile;
+  d.ntok = min(kTokTile, n_e - d.chunk * kTokTile);
+  if (P.mode == kModeGateUp) {
+    d.rb0 = d.bp;
+    d.rb1 = P.rows_half / kRowBlock + d.bp;
+  } else {
+    d.rb0 = 2 * d.bp;
+    d.rb1 = 2 * d.bp + 1;
+  }
+  return d;
+}
+
+__global__ void __launch_bounds__(kGThreads, 1)
+grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ CUtensorMap xmap) {
+  extern __shared__ __align__(1024) uint8_t gsmem_raw[];
+  // the dynamic shared window is only guaranteed 16-byte aligned: align the carve-out by hand
+  GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0) {
+    for (int i = 0; i < kGStages; ++i) {
+      tc::mbar_init(&s.full[i], 1);
+      tc::mbar_init(&s.empty[i], 8 + 1);       // 8 dequant warps + the MMA commit
+    }
+    for (int i = 0; i < 2; ++i) { tc::mbar_init(&s.afull[i], 8); tc::mbar_init(&s.aempty[i], 1); }
+    tc::mbar_init(&s.dfull, 1);
+    tc::mbar_init(&s.dempty, 4);
+    for (int i = 0; i < 4; ++i) { tc::mbar_init(&s.tq_full[i], 1); tc::mbar_init(&s.tq_empty[i], 1 + 4 + 8); }
+    tc::mbar_init(&s.drain, 1);
+    s.abort = 0;
+    tc::fence_barrier_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&xmap) : "memory");
+  }
+  if (warp == 1) {
+    tc::tmem_alloc<kGTmemCols>(&s.tmem_base);
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abort = &s.abort;
+  const int total = *P.ntiles;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    const uint64_t pol_w = tc::policy_evict_last();   // weights are reused across token chunks
+    int it = 0;
+    for (int n = 0;; ++n) {
+      int t = 0;
+      if (lane == 0) t = atomicAdd(P.ctl + kCtlClaim, 1);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      const bool stop = t >= total || *abort;
+      const int q = n & 3;
+      if (!gwait(&s.tq_empty[q], ((n >> 2) & 1) ^ 1, abort)) {
+        if (lane == 0) report_status(P.ctl, MOE_ERR_TIMEOUT, 21);
+        break;
+      }
+      if (lane == 0) {
+        s.tq[q] = stop ? -1 : P.tile_list[t];
+        tc::mbar_arrive(&s.tq_full[q]);
+      }
+      if (stop) break;
+      const TileDesc d = describe(P, P.tile_list[t]);
+      const uint8_t* wb = P.w + (size_t)d.slot * P.w_stride;
+      const uint16_t* sb = P.s + (size_t)d.slot * P.s_stride;
+      bool ok = true;
+      for (int g = 0; g < P.G; ++g, ++it) {
+        const int st = it % kGStages;
+        if (!gwait(&s.empty[st], ((it / kGStages) & 1) ^ 1, abort)) { ok = false; break; }
+        if (lane == 0) {
+          GStage& S = s.st[st];
+          tc::mbar_arrive_expect_tx(&s.full[st], 2 * kBBoxBytes + 2 * 8192 + 2 * 256);
+          tma_load_2d(S.b[0], &xmap, g * 128, d.p0, &s.full[st]);
+          tma_load_2d(S.b[1], &xmap, g * 128 + 64, d.p0, &s.full[st]);
+          const size_t t0 = d.rb0 * P.G + g, t1 = d.rb1 * P.G + g;
+          tc::bulk_g2s(S.w[0], wb + t0 * kTileBytes, 8192, &s.full[st], pol_w);
+          tc::bulk_g2s(S.w[1], wb + t1 * kTileBytes, 8192, &s.full[st], pol_w);
+          tc::bulk_g2s(S.sc[0], sb + t0 * kRowBlock, 256, &s.full[st], pol_w);
+          tc::bulk_g2s(S.sc[1], sb + t1 * kRowBlock, 256, &s.full[st], pol_w);
+        }
+      }
+      if (!ok) {
+        if (lane == 0) report_status(P.ctl, MOE_ERR_TIMEOUT, 22);
+        if (lane == 0) s.abort = 1;
+        break;
+      }
+    }
+    if (lane == 0) {   // no copy may still be landing when the CTA leaves
+      const int n = it < kGStages ? it : kGStages;
+      for (int i = 0; i < n; ++i) {
+        const int j = it - 1 - i;
+        volatile int never = 0;
+        tc::mbar_wait(&s.full[j % kGStages], (j / kGStages) & 1, &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int it = 0, a_it = 0;
+      for (int n = 0;; ++n) {
+        const int q = n & 3;
+        if (!tc::mbar_wait(&s.tq_full[q], (n >> 2) & 1, abort)) { report_status(P.ctl, MOE_ERR_TIMEOUT, 23); break; }
+        const int packed = s.tq[q];
+        tc::mbar_arrive(&s.tq_empty[q]);
+        if (packed < 0) break;
+        const TileDesc d = describe(P, packed);
+        const int nmma = (d.ntok + 15) & ~15;
+        const uint32_t idesc = tc::idesc_bf16_f32(128, nmma);
+        if (!tc::mbar_wait(&s.dempty, (n & 1) ^ 1, abort)) { report_status(P.ctl, MOE_ERR_TIMEOUT, 24); break; }
+        tc::tc_fence_after();
+        bool ok = true;
+        for (int g = 0; g < P.G; ++g, ++it, ++a_it) {
+          const int st = it % kGStages, ab = a_it & 1;
+          if (!tc::mbar_wait(&s.full[st], (it / kGStages) & 1, abort) ||
+              !tc::mbar_wait(&s.afull[ab], (a_it >> 1) & 1, abort)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t bbase = tc::smem_u32(s.st[st].b[0]);
+          const uint32_t a0 = tmem + kGA + ab * 128, a1 = a0 + 64;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t baddr = bbase + (kk >> 2) * kBBoxBytes + (kk & 3) * 32;
+            const uint64_t bdesc = tc::smem_desc(baddr, 16, 1024, 2);
+            const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
+            tc::mma_ts(tmem + kGD0, a0 + kk * 8, bdesc, idesc, acc);
+            tc::mma_ts(tmem + kGD1, a1 + kk * 8, bdesc, idesc, acc);
+          }
+          tc::mma_commit(&s.aempty[ab]);
+          tc::mma_commit(&s.empty[st]);
+        }
+        if (!ok) {
+          report_status(P.ctl, MOE_ERR_TIMEOUT, 25);
+          s.abort = 1;
+          break;
+        }
+        tc::mma_commit(&s.dfull);
+      }
+      tc::mma_commit(&s.drain);
+      volatile int never = 0;
+      tc::mbar_wait(&s.drain, 0, &never);
+    }
+    __syncwarp();
+  } else if (warp >= kGDq0) {
+    // ---------------------------------------------------------------- dequantisers -> TMEM
+    const int quarter = warp & 3, blk = (warp - kGDq0) >> 2;     // block 0 or 1 of the pair
+    const int r = quarter * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + kGA + blk * 64;
+    const __nv_bfloat162 off136 = __floats2bfloat162_rn(136.f, 136.f);
+    int it = 0, a_it = 0;
+    for (int n = 0;; ++n) {
+      const int q = n & 3;
+      if (!gwait(&s.tq_full[q], (n >> 2) & 1, abort)) break;
+      const int packed = s.tq[q];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s.tq_empty[q]);
+      if (packed < 0) break;
+      bool ok = true;
+      for (int g = 0; g < P.G; ++g, ++it, ++a_it) {
+        const int st = it % kGStages, ab = a_it & 1;
+        if (!gwait(&s.full[st], (it / kGStages) & 1, abort)) { ok = false; break; }
+        const uint8_t* wsrc = s.st[st].w[blk];
+        uint4 c[4];
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) c[kq] = *reinterpret_cast<const uint4*>(wsrc + kq * 2048 + r * 16);
+        const uint32_t sbits = s.st[st].sc[blk][r];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&s.empty[st]);
+        const uint32_t s2u = sbits | (sbits << 16);
+        const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+        if (!gwait(&s.aempty[ab], ((a_it >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+        tc::tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t words[8] = {c[2 * h].x, c[2 * h].y, c[2 * h].z, c[2 * h].w,
+                                     c[2 * h + 1].x, c[2 * h + 1].y, c[2 * h + 1].z, c[2 * h + 1].w};
+          uint32_t v[32];
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const uint32_t t = ((words[w] >> (4 * p)) & 0x000F000Fu) | 0x43004300u;
+              const __nv_bfloat162 qv = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&t), off136);
+              const __nv_bfloat162 wv = __hmul2(qv, s2);
+              v[w * 4 + p] = *reinterpret_cast<const uint32_t*>(&wv);
+            }
+          tc::tmem_st32(trow + ab * 128 + h * 32, v);
+        }
+        tc::tmem_wait_st();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&s.afull[ab]);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int n = 0;; ++n) {
+      const int q = n & 3;
+      if (!gwait(&s.tq_full[q], (n >> 2) & 1, abort)) break;
+      const int packed = s.tq[q];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s.tq_empty[q]);
+      if (packed < 0) break;
+      const TileDesc d = describe(P, packed);
+      if (!gwait(&s.dfull, n & 1, abort)) break;
+      tc::tc_fence_after();
+      for (int c0 = 0; c0 < d.ntok; c0 += 32) {
+        uint32_t v0[32], v1[32];
+        tmem_ld32(trow + kGD0 + c0, v0);
+        tmem_ld32(trow + kGD1 + c0, v1);
+        tc::tmem_wait_ld();
+        const int cn = min(32, d.ntok - c0);
+        if (P.mode == kModeGateUp) {
+          const size_t col = d.bp * kRowBlock + r;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < cn) {
+              const float g = __uint_as_float(v0[j]), u = __uint_as_float(v1[j]);
+              const float h = g / (1.f + expf(-g)) * u;
+              P.out[(size_t)(d.p0 + c0 + j) * P.out_ld + col] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
+            }
+          }
+        } else {
+          const size_t col0 = d.rb0 * kRowBlock + r, col1 = d.rb1 * kRowBlock + r;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            if (j < cn) {
+              const int pos = d.p0 + c0 + j;
+              const float w = P.wts[P.perm[pos]];
+              uint16_t* o = P.out + (size_t)pos * P.out_ld;
+              o[col0] = __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(v0[j])));
+              o[col1] = __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(v1[j])));
+            }
+          }
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&s.dempty);
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc<kGTmemCols>(tmem);
+  }
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(P.ctl + kCtlDone, 1) == (int)gridDim.x - 1) {
+      __threadfence();
+      P.ctl[kCtlClaim] = 0;
+      P.ctl[kCtlDone] = 0;
+      __threadfence();
+    }
+  }
+}
+
+// One block per expert: writes that expert's tiles (chunk-major, block pair minor) at its
+// prefix offset in the list, and block 0 writes the total.
+__global__ void __launch_bounds__(256) tile_list_kernel(const int32_t* __restrict__ counts, int E,
+                                                        const int32_t* __restrict__ table, int pairs,
+                                                        int32_t* __restrict__ list, int32_t* __restrict__ total) {
+  const int e = blockIdx.x;
+  __shared__ int base, mine;
+  if (threadIdx.x == 0) {
+    int b = 0, tot = 0;
+    for (int x = 0; x < E; ++x) {
+      const int n = (slot_of(table, x) >= 0) ? (counts[x] + kTokTile - 1) / kTokTile * pairs : 0;
+      if (x < e) b += n;
+      if (x == e) mine = n;
+      tot += n;
+    }
+    base = b;
+    if (e == 0) *total = tot;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < mine; i += blockDim.x) {
+    const int chunk = i / pairs, bp = i % pairs;
+    list[base + i] = (e << 24) | (chunk << 12) | bp;
+  }
+}
+
+// out[t] = bf16( acc + sum_j yw[inv[t][j]] ) with yw already weighted (bf16), fixed j order.
+__global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __restrict__ yw,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ inv,
+                                                           const int32_t* __restrict__ table, int H, int k,
+                                                           float* __restrict__ acc, bool accumulate,
+                                                           uint16_t* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int n0 = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
+  if (n0 >= H) return;
+  float v[8];
+  float* accp = acc + (size_t)t * H + n0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = accumulate ? accp[i] : 0.f;
+  for (int j = 0; j < k; ++j) {
+    if (slot_of(table, idx[(size_t)t * k + j]) < 0) continue;
+    const uint4 y = *reinterpret_cast<const uint4*>(yw + (size_t)inv[(size_t)t * k + j] * H + n0);
+    const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] += bf16_bits_to_float(yy[i] & 0xffffu);
+      v[2 * i + 1] += bf16_bits_to_float(yy[i] >> 16);
+    }
+  }
+  if (out) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      pk[i] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + n0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    if (accumulate)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) accp[i] = 0.f;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) accp[i] = v[i];
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+  if (g_encode) return MOE_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return MOE_OK;
+}
+
+// 2-D map over a row-major bf16 matrix [rows][cols]: box = 64 columns x 128 rows, 128B swizzle.
+int make_rows_map(CUtensorMap* map, const void* base, int rows, int cols) {
+  if (int rc = get_encode()) return rc;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kTokTile};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOE_OK;
+}
+
+int g_sms = 0;
+int sm_count() {
+  if (!g_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_sms <= 0) g_sms = 148;
+  }
+  return g_sms;
+}
+
+int launch_gemm(const GParams& P, const CUtensorMap& map, int max_tiles, cudaStream_t s) {
+  const size_t smem = sizeof(GSmem) + 1024;
+  static bool attr = false;
+  if (!attr) {
+    if (int rc = check_cuda(cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem), "grouped GEMM: smem attribute"))
+      return rc;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(std::max(1, std::min(sm_count(), max_tiles)));
+  cfg.blockDim = dim3(kGThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel, P, map);
+  note_launch();
+  return check_cuda(e, "grouped_gemm_kernel launch");
+}
+
+}  // namespace
+
+bool ffn_grouped_supported(const FfnArgs& a) {
+  return a.T >= 1 && a.E <= kMaxExperts && a.H % 256 == 0 && a.I % kRowBlock == 0 && (size_t)a.T * a.k < (1u << 20) &&
+         (a.T * a.k + kTokTile - 1) / kTokTile < 4096;
+}
+
+int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
+  const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
+  const int Tk = a.T * a.k;
+  int32_t* counts = reinterpret_cast<int32_t*>(a.ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(a.ws + L.offsets);
+  int32_t* perm = reinterpret_cast<int32_t*>(a.ws + L.perm);
+  int32_t* inv = reinterpret_cast<int32_t*>(a.ws + L.inv);
+  int32_t* tiles = reinterpret_cast<int32_t*>(a.ws + L.tiles);      // [0]: gate/up total, [1]: down total
+  int32_t* list_gu = reinterpret_cast<int32_t*>(a.ws + L.tile_list);
+  int32_t* list_dn = list_gu + L.tile_list_len;
+  uint16_t* xp = reinterpret_cast<uint16_t*>(a.ws + L.xp);
+  uint16_t* hp = reinterpret_cast<uint16_t*>(a.ws + L.hp);
+  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // weighted y, bf16
+  int* ctl = reinterpret_cast<int*>(a.ws + L.status);
+
+  if (int rc = launch_permute(a.idx, a.T, a.k, a.E, counts, offsets, perm, inv,
+                              reinterpret_cast<int32_t*>(a.ws + L.perm_scratch), s))
+    return rc;
+  if (int rc = launch_gather_rows(a.x, perm, Tk, a.k, a.H, xp, s)) return rc;
+  const int IB = a.I / kRowBlock, HP = a.H / 256;
+  tile_list_kernel<<<a.E, 256, 0, s>>>(counts, a.E, a.slot, IB, list_gu, tiles + 0);
+  if (int rc = check_launch("tile_list_kernel")) return rc;
+  tile_list_kernel<<<a.E, 256, 0, s>>>(counts, a.E, a.slot, HP, list_dn, tiles + 1);
+  if (int rc = check_launch("tile_list_kernel")) return rc;
+  const int max_chunks = (Tk + kTokTile - 1) / kTokTile + a.E;
+
+  CUtensorMap xmap, hmap;
+  if (int rc = make_rows_map(&xmap, xp, Tk, a.H)) return rc;
+  if (int rc = make_rows_map(&hmap, hp, Tk, a.I)) return rc;
+
+  GParams P{};
+  P.w = a.w13; P.s = a.s13;
+  P.w_stride = (size_t)2 * a.I * a.H / 2; P.s_stride = (size_t)2 * a.I * (a.H / kGroup);
+  P.K = a.H; P.G = a.H / kGroup; P.rows_half = a.I; P.mode = kModeGateUp;
+  P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
+  P.perm = perm; P.wts = a.wts; P.out = hp; P.out_ld = a.I; P.Tk = Tk; P.ctl = ctl;
+  if (int rc = launch_gemm(P, xmap, max_chunks * IB, s)) return rc;
+
+  P.w = a.w2; P.s = a.s2;
+  P.w_stride = (size_t)a.H * a.I / 2; P.s_stride = (size_t)a.H * (a.I / kGroup);
+  P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
+  P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;
+  if (int rc = launch_gemm(P, hmap, max_chunks * HP, s)) return rc;
+
+  dim3 grid(a.T, ceil_div(a.H, 256 * 8));
+  combine_bf16_kernel<<<grid, 256, 0, s>>>(yw, a.idx, inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
+                                           a.accumulate, a.out);
+  return check_launch("combine_bf16_kernel");
+}
+
+}  // namespace moe
