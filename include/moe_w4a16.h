@@ -71,6 +71,11 @@ const char* moe_last_error_string(void);
  * captured) in this process so far; a diagnostic for benchmarks. */
 unsigned long long moe_launch_count(void);
 
+/* Diagnostics: when dev_buffer is non-NULL, the fused decode kernel records per-CTA
+ * timestamps (%globaltimer, 64 unsigned 64-bit slots per CTA, one row per CTA) into it; NULL
+ * turns recording off. The buffer must hold 64 * (number of SMs) slots. */
+void moe_debug_set_decode_trace(void* dev_buffer);
+
 /* Bytes of packed codes of one N x K matrix (N*K/2) and number of its bf16 scales
  * (N*K/128). Return 0 when N or K is not a positive multiple of 128. */
 size_t moe_packed_bytes(int N, int K);

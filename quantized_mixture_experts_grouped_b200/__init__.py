@@ -42,6 +42,7 @@ def _load() -> ctypes.CDLL:
         "moe_packed_layout_version": ([], I),
         "moe_last_error_string": ([], c.c_char_p),
         "moe_launch_count": ([], c.c_ulonglong),
+        "moe_debug_set_decode_trace": ([P], None),
         "moe_packed_bytes": ([I, I], Z),
         "moe_scales_count": ([I, I], Z),
         "moe_quantize_pack": ([P, I, I, I, P, P, P], I),

@@ -18,13 +18,18 @@ pytestmark = pytest.mark.gpu
 
 q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
 
-FFN_PATHS = ["simple", "decode"]
+FFN_PATHS = ["simple", "decode", "grouped"]
 
 
 def _supported(path, T, k):
-    """The fused decode path takes small batches only (T <= 32 and T*k <= 256)."""
-    if path == "decode" and not (1 <= T <= 32 and T * k <= 256):
+    """The fused decode path takes small batches only (T <= 16 and T*k <= 256)."""
+    if path == "decode" and not (1 <= T <= 16 and T * k <= 256):
         pytest.skip("fused decode path is for small batches")
+
+
+def _supported_h(path, H):
+    if path == "grouped" and H % 256:
+        pytest.skip("grouped GEMM pairs 128-row blocks of W2: H must be a multiple of 256")
 
 
 def _ws(T, H, I, E, k):
@@ -151,6 +156,7 @@ def test_permute_bit_exact(T, E, k):
 
 def _run_ffn(layer: Layer, path: str, out=None, slot=None):
     _supported(path, layer.T, layer.wl.k)
+    _supported_h(path, layer.wl.H)
     d = layer.to_device()
     wl = layer.wl
     ws = _ws(layer.T, wl.H, wl.I, wl.E, wl.k)
@@ -163,7 +169,7 @@ def _run_ffn(layer: Layer, path: str, out=None, slot=None):
 
 
 @pytest.mark.parametrize("path", FFN_PATHS)
-@pytest.mark.parametrize("T", [4, 1, 17, 64])
+@pytest.mark.parametrize("T", [4, 1, 16, 17, 64])
 def test_ffn_tiny_shapes(path, T):
     layer = Layer(mi.WORKLOADS["tiny"], T=T)
     out, _ = _run_ffn(layer, path)
@@ -172,7 +178,7 @@ def test_ffn_tiny_shapes(path, T):
 
 @pytest.mark.parametrize("path", FFN_PATHS)
 def test_ffn_edge_cases(path):
-    wl = mi.Workload("edge", H=384, I=256, E=8, k=3, T=37)
+    wl = mi.Workload("edge", H=512, I=384, E=8, k=3, T=37)
     g = np.random.default_rng(2)
     # one expert takes every token (its logit dominates), two experts get none
     l = g.standard_normal((wl.T, wl.E)).astype(np.float32)
@@ -199,7 +205,7 @@ def test_ffn_k_equals_e(path):
 @pytest.mark.parametrize("path", FFN_PATHS)
 def test_ffn_edge_cases_small_batch(path):
     """Decode-sized batch: one expert takes every token, two get none, one all-zero group."""
-    wl = mi.Workload("edge_small", H=384, I=256, E=8, k=3, T=21)
+    wl = mi.Workload("edge_small", H=512, I=384, E=8, k=3, T=13)
     g = np.random.default_rng(3)
     l = g.standard_normal((wl.T, wl.E)).astype(np.float32)
     l[:, 2] += 100.0
@@ -211,10 +217,11 @@ def test_ffn_edge_cases_small_batch(path):
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
 
 
-@pytest.mark.parametrize("path", ["auto", "decode", "simple"])
-@pytest.mark.parametrize("T", [1, 5, 16])
+@pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped"])
+@pytest.mark.parametrize("T", [1, 5, 16, 300])
 def test_layer_call_routes_and_runs(path, T):
     """moe_w4a16_layer: routing (in-kernel on the fused path) + FFN in one call."""
+    _supported(path, T, 4)
     wl = mi.Workload("layer", H=512, I=256, E=16, k=4, T=T)
     layer = Layer(wl, layer=1, step=T)
     d = layer.to_device()
@@ -270,7 +277,7 @@ def test_ffn_large_expert_full_size_sampled(path):
 
 @pytest.mark.parametrize("path", FFN_PATHS)
 def test_ffn_deterministic_and_slot_indirection(path):
-    layer = Layer(mi.WORKLOADS["tiny"], T=19)
+    layer = Layer(mi.WORKLOADS["tiny"], T=15)
     _supported(path, layer.T, layer.wl.k)
     a, _ = _run_ffn(layer, path)
     b, _ = _run_ffn(layer, path)
