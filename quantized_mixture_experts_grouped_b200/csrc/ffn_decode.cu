@@ -81,7 +81,9 @@ struct DecParams {
 };
 
 // trace slots per CTA (64 x u64): 0 start, 1 plan done, 2 first tile issued, 3 producer done,
-// 4 epilogue done, 5 end, 8.. epilogue finish time of the i-th unit
+// 4 epilogue done, 5 end, 8..15 epilogue finish time of the i-th unit, 16..47 dequant group 0
+// (4 per tile: stage ready, stage read, A buffer free, TMEM written), 48..55 plan phases,
+// 56..63 MMA issue of the first 8 tiles
 __device__ __forceinline__ void trace_at(const DecParams& P, int slot) {
   if (P.trace) P.trace[blockIdx.x * 64 + slot] = tc::globaltimer();
 }
@@ -248,8 +250,10 @@ __device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
       if (n < P.T) xv[i] = __ldg(reinterpret_cast<const uint4*>(P.x + (size_t)n * P.H) + kc);
     }
   }
+  if (tid == 0) trace_at(P, 48);
   if (P.logits) {
     if (warp < P.T) route_token(s, P, warp, lane);
+    if (tid == 0) trace_at(P, 49);
   } else {
     for (int i = tid; i < Tk; i += kThreads) {
       s.idx[i] = P.idx_in[i];
@@ -272,6 +276,7 @@ __device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
     }
   }
   __syncthreads();
+  if (tid == 0) trace_at(P, 50);
   if (P.logits && P.idx_out && blockIdx.x == 0)
     for (int i = tid; i < Tk; i += kThreads) {
       P.idx_out[i] = s.idx[i];
@@ -289,6 +294,7 @@ __device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
     if (e >= 0 && lower == 0) s.wcount[warp][e] = __popc(same);
   }
   __syncthreads();
+  if (tid == 0) trace_at(P, 51);
   for (int x = tid; x < E; x += kThreads) {
     int c = 0;
     for (int w = 0; w < 8; ++w) c += s.wcount[w][x];
@@ -321,6 +327,7 @@ __device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
     }
   }
   __syncthreads();
+  if (tid == 0) trace_at(P, 52);
   for (int i = tid; i < s.nact * kMaxT; i += kThreads) s.posof[i / kMaxT][i % kMaxT] = -1;
   __syncthreads();
   if (tid < Tk && e >= 0) {
@@ -344,6 +351,7 @@ __device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
     s.tokmask[a] = m;
   }
   __syncthreads();
+  if (tid == 0) trace_at(P, 53);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ DecParams P) {
@@ -454,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         for (int ti = 0; ti < U.ntile; ++ti, ++a_it) {
           const int ab = a_it % kABufs;
           if (!tc::mbar_wait(&s.afull[ab], (a_it / kABufs) & 1, abort)) { ok = false; report_abort(s, P, kSiteABuf); break; }
+          if (a_it < 8) trace_at(P, 56 + a_it);
           const uint32_t a = tmem + kAColBase + ab * 64;
           if (U.type == 0) {
             tc::tc_fence_after();
@@ -501,16 +510,20 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         if ((it & 1) != grp) continue;
         const int st = it % kStages;
         if (!warp_wait(&s.full[st], (it / kStages) & 1, abort)) { ok = false; break; }
+        const bool tr = (warp == kDqWarp0 && lane == 0 && it < 16);
+        if (tr) trace_at(P, 16 + (it >> 1) * 4);
         uint4 c[4];
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) c[kq] = *reinterpret_cast<const uint4*>(s.stage[st] + kq * 2048 + r * 16);
         const uint32_t sb = s.scale[st][r];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&s.empty[st]);
+        if (tr) trace_at(P, 17 + (it >> 1) * 4);
         const uint32_t s2u = sb | (sb << 16);
         const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
         const int ab = it % kABufs;
         if (!warp_wait(&s.aempty[ab], ((it / kABufs) & 1) ^ 1, abort)) { ok = false; break; }
+        if (tr) trace_at(P, 18 + (it >> 1) * 4);
         tc::tc_fence_after();
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -529,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
           tc::tmem_st32(taddr_row + ab * 64 + h * 32, v);
         }
         tc::tmem_wait_st();
+        if (tr) trace_at(P, 19 + (it >> 1) * 4);
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&s.afull[ab]);
