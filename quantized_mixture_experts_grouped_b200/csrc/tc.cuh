@@ -38,29 +38,43 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// One bounded try: the thread may be suspended by the hardware (not spinning) for up to
+// kSuspendNs while the phase is incomplete.
+constexpr uint32_t kSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
 
+// SM clock cycles after which a wait gives up (about 2 s at the B200's 1.97 GHz peak clock;
+// longer at lower clocks). The SM-local cycle counter is cheap to read, unlike %globaltimer.
+constexpr long long kWaitTimeoutCycles = 4000000000ll;
+
 // Waits until the phase with the given parity has completed. Returns false on timeout (after
-// raising *abort) or when *abort is already raised.
+// raising *abort) or when *abort is already raised. The abort flag and the clock are looked at
+// every 64 tries only; each try may itself sleep in hardware (see mbar_try_wait).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  while (true) {
+  long long t0 = 0;
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > kWaitTimeoutNs) {
-      *abort = 1;
-      return false;
+    if ((i & 63) == 0) {
+      if (*abort) return false;
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitTimeoutCycles) {
+        *abort = 1;
+        return false;
+      }
     }
   }
 }
