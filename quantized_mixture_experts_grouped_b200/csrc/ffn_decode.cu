@@ -4,118 +4,92 @@
 // grouped MoE kernels; the router's top-k is unchanged).
 //
 // A decode batch (T <= 16 tokens) reads every selected expert's packed weights exactly once, so
-// the layer is bound by HBM bandwidth on those bytes plus the latency of every dependent step.
-// The kernel is shaped to keep that chain short:
+// the layer is bound by HBM bandwidth on those bytes plus the latency of its dependent steps.
+// On B200 a CTA only streams near its share of HBM bandwidth when it moves weights in large
+// bulk copies (tens of KB each) with several in flight, so the work is cut into byte-balanced
+// contiguous runs of packed tiles rather than into whole experts or feature slices:
 //  * every CTA routes the batch itself (warp top-k; the renormalised weights are a softmax over
-//    the k chosen logits, which equals the full softmax renormalised) and builds the grouping
-//    with a presence bitmap and shared-memory atomics (constant depth); the batch's activations
-//    are staged once in shared memory as the B operand of every gate/up MMA (all T tokens are
-//    MMA columns; a column whose token is not routed to the expert is computed and ignored);
-//  * a unit is (routed expert, 64 intermediate features); CTA c takes units c, c+G, c+2G, ...
-//    A unit needs no other CTA: gate and up rows of its 64 features form one 128-row MMA over
-//    all of H, the CTA turns the accumulators into h = w * silu(g) * u itself (gate and up
-//    rows meet through shared memory), and multiplies h by the matching 64-wide column slice
-//    of W2 for every row of H. All units of a CTA accumulate into one tensor-memory
-//    accumulator, so the router-weighted sum over experts happens inside the MMA;
-//  * warp 0 streams the unit's int4 weights + bf16 scales into an 8-stage shared-memory ring
-//    with bulk async copies (TMA, evict-first in L2);
-//  * warps 6..13 dequantise in two groups that take alternate stages: a thread owns one weight
+//    the k chosen logits, which equals the full softmax renormalised), lists the selected
+//    experts in ascending id, and stages the activations in shared memory as the B operand of
+//    every gate/up MMA (all T tokens are MMA columns; columns of unrouted tokens are ignored);
+//  * phase 1 (gate/up): the selected experts' W13 tiles, expert by expert in stored order, are
+//    split evenly over the CTAs. A CTA accumulates each 128-row block it touches over its part
+//    of K and writes the fp32 partial. The CTA that completes the last partial of a feature
+//    block (gate rows f..f+127 and up rows I+f..I+f+127) sums the partials in CTA order and
+//    writes h = w_router * silu(gate) * up in bf16 (zero for tokens not routed to the expert);
+//  * phase 2 (down): W2 tiles ordered (output row block, expert, K group) are split the same
+//    way. A CTA accumulates one output row block over all experts and K groups it covers, so
+//    the router-weighted sum over experts happens inside the tensor-memory accumulator; the h
+//    operand of each tile arrives with it. The CTA completing an output block's last partial
+//    sums the partials in CTA order and writes the bf16 outputs. Down weights are prefetched
+//    while phase 1 still runs; only their h operands wait until every feature block is done;
+//  * warp 0 streams int4 codes + bf16 scales in copies of up to four tiles (32 KB) into a ring
+//    of shared-memory stages (TMA bulk copies, evict-first in L2); its lanes issue the copies
+//    of a stage side by side, since each issuing thread pays a fixed latency per copy;
+//  * warps 6..13 dequantise in two groups that take alternate tiles: a thread owns one weight
 //    row and writes bf16 (q * s, one rounding) straight into TENSOR MEMORY (tcgen05.st) as the
 //    A operand of tcgen05.mma - the bf16 weights never pass through shared memory;
-//  * one thread of warp 1 issues tcgen05.mma (M = 128 weight rows, N = 16 tokens, K = 16);
-//  * warps 2..5 run the epilogues: h for each unit, then the CTA's partial output;
-//  * a grid-wide barrier (sense-reversing, bounded) separates the units from the final
-//    reduction, where every CTA sums one slice of the per-CTA partials in a fixed order and
-//    writes bf16 outputs. Results are deterministic run to run.
-// Every wait is bounded; on a timeout the kernel records MOE_ERR_TIMEOUT in the workspace,
-// drains its own copies and MMAs, frees its tensor memory and exits.
-#include <algorithm>
-
-#include "common.cuh"
-#include "tc.cuh"
+//  * one thread in each of warps 1 and 14 issues tcgen05.mma (M = 128 weight rows, N = 16
+//    tokens, K = 16) for alternate tiles into its own accumulators: with N this small an MMA
+//    costs its issuing thread about as much as a full-width one, so two issuers double the
+//    rate at which tiles are consumed;
+//  * warps 2..5 drain accumulators, add the two issuers' parts, write partials and run the
+//    reductions above.
+// Every reduction runs in a fixed order, so results are identical run to run. Every wait is
+// bounded; on a timeout the kernel records MOE_ERR_TIMEOUT in the workspace, drains its own
+// copies and MMAs, frees its tensor memory and exits (the workspace must then be re-initialised).
+#include "decode_common.cuh"
 
 namespace moe {
+namespace dec {
 
-__device__ __forceinline__ uint32_t route_key_d(uint32_t bits, int e) {
-  bits &= 0xffffu;
-  if (bits == 0x8000u) bits = 0;
-  const uint32_t ord = (bits & 0x8000u) ? (~bits & 0xffffu) : (bits | 0x8000u);
-  return (ord << 16) | (0xffffu - (uint32_t)e);
+unsigned long long* g_trace = nullptr;
+int g_num_sms = 0;
+
+int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
 }
 
 namespace {
 
-constexpr int kStages = 8;
-constexpr int kABufs = 3;
-constexpr int kMaxTk = 256;
-constexpr int kMaxT = 16;
-constexpr int kN = 16;                    // MMA N: the batch's tokens (<= 16)
-constexpr int kIF = 64;                   // intermediate features per unit
-constexpr int kMaxHB = 16;                // H <= 2048: one accumulator column block per 128 rows
-constexpr int kMaxGrid = 160;
-constexpr int kThreads = 448;             // 14 warps
+constexpr int kN = 16;                     // MMA N: the batch's tokens (<= 16)
+constexpr int kMaxStages = 4;
+constexpr int kABufs = 4;                  // dequantised tiles in tensor memory (64 columns each)
+constexpr int kIssuers = 2;                // MMA-issuing threads (one per warp)
+constexpr int kAcc = 8;                    // accumulators per issuer (16 columns each)
+constexpr int kThreads = 480;              // 15 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kEpiWarp0 = 2;              // warps 2..5
-constexpr int kDqWarp0 = 6;               // warps 6..13: two groups of four
+constexpr int kIssuerWarp0 = 1;
+constexpr int kEpiWarp0 = 2;               // warps 2..5
+constexpr int kDqWarp0 = 6;                // warps 6..13: two groups of four
+constexpr int kDqWarpsPerGroup = 4;
+constexpr int kIssuerWarp1 = 14;
 constexpr int kTmemCols = 512;
-constexpr int kAColBase = 0;              // 3 A buffers x 64 columns
-constexpr int kDguCol = 192;              // gate/up accumulators: 2 x kN columns
-constexpr int kDhCol = 256;               // partial output: kMaxHB x kN columns
-constexpr unsigned kFull = 0xffffffffu;
-constexpr int kCtlBarCount = kCtlDecode;      // grid barrier arrivals
-constexpr int kCtlBarGen = kCtlDecode + 1;    // grid barrier generation
-
-enum { kSiteStage = 2, kSiteABuf = 3, kSiteB = 4, kSiteD = 5, kSiteGrid = 6, kSiteDrain = 7, kSiteOver = 8 };
-
-struct DecParams {
-  const uint16_t* x; const uint16_t* logits; const int32_t* idx_in; const float* wts_in;
-  int T, H, I, E, k;
-  const uint8_t* w13; const uint16_t* s13; const uint8_t* w2; const uint16_t* s2;
-  const int32_t* slot;
-  int32_t* idx_out; float* wts_out;
-  uint16_t* out; float* acc; int accumulate;
-  int* ctl;
-  float* ypart;                 // [gridDim][T][H] per-CTA partial outputs
-  unsigned long long* trace;    // optional per-CTA timestamps (diagnostics), null in normal use
-};
-
-// trace slots per CTA (64 x u64, %globaltimer): 0 start, 1 plan done, 2 first copy issued,
-// 3 producer done, 4 epilogue done, 5 grid barrier passed, 6 end
-__device__ __forceinline__ void trace_at(const DecParams& P, int slot) {
-  if (P.trace) P.trace[blockIdx.x * 64 + slot] = tc::globaltimer();
-}
+constexpr int kAColBase = 0;
+constexpr int kAccCol = kABufs * 64;
+constexpr int kHTile = 2048;               // one 8-token row group of a 128-wide h tile (bf16)
+constexpr int kStageH = 2 * kTilesPerStage * kHTile;
+constexpr int kStageBytes = kStageW + kStageS + kStageH;
 
 struct __align__(128) DecSmem {
-  uint8_t stage[kStages][8192];
-  uint16_t scale[kStages][128];
-  uint8_t bdown[2][kN * kIF * 2];           // h of a unit: B operand of the down MMA (2 KB each)
-  float gx[kIF][kN];                        // gate accumulators handed to the up-row warps
-  float red[kThreads];                      // final-reduction scratch
-  int idx[kMaxTk];
-  float wts[kMaxTk];
-  uint32_t present[kMaxExperts / 32];
-  int act[kMaxExperts];
-  int aidx[kMaxExperts];
-  uint32_t tokmask[kMaxExperts];
-  float wtok[kMaxExperts][kMaxT];           // router weight of (active expert, token), 0 if not routed
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kMaxStages], empty[kMaxStages], hfull[kMaxStages];
   uint64_t afull[kABufs], aempty[kABufs];
-  uint64_t gfull[2], gempty[2];             // gate/up accumulators
-  uint64_t bfull[2], bempty[2];             // h operand
-  uint64_t hfull, drain;
+  uint64_t accfull[kIssuers][kAcc], accempty[kIssuers][kAcc];
+  uint64_t drain[kIssuers];
+  RouteSmem rs;
+  float wsel[kMaxT];
   uint32_t tmem_base;
-  int nact;
   int abort;
-  int over;
-  // followed in dynamic shared memory by the activations: kN rows x H, no-swizzle K-major
+  int epi_dec;
+  // followed in dynamic shared memory by the activations (kN rows x H, no-swizzle K-major)
+  // and by the stage ring
 };
-
-// Every lane waits (each gets the barrier's acquire); the outcome is made warp-uniform so that
-// a timeout can never leave the lanes of one warp on different paths.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = tc::mbar_wait(bar, parity, abort);
-  return __all_sync(kFull, ok);
-}
 
 __device__ __forceinline__ void report_abort(DecSmem& s, const DecParams& P, int site) {
   s.abort = 1;
@@ -142,146 +116,46 @@ __device__ __forceinline__ void dequant_half(uint4 a, uint4 b, __nv_bfloat162 s2
   tc::tmem_st32(taddr, v);
 }
 
-// Element (n, k) of a kN-row, K-major operand without swizzle: 8x16-byte core matrices.
+// Element (n, k) of the kN-row, K-major activation operand without swizzle: 8x16-byte core
+// matrices, K-direction core stride 256 bytes, row-group stride 128 bytes.
 __device__ __forceinline__ uint32_t kmajor_off(int n, int k) {
   return (uint32_t)(((k >> 3) * (kN / 8) + (n >> 3)) * 128 + (n & 7) * 16 + (k & 7) * 2);
 }
 
-// Routes token t with one warp (same selection rule as route_kernel): writes s.idx / s.wts and
-// marks the chosen experts in the presence bitmap. The chosen logits are decoded back from the
-// winning keys; the renormalised weight of choice j is exp(l_j - l_max) / sum over the k chosen.
-__device__ void route_token(DecSmem& s, const DecParams& P, int t, int lane) {
-  const int E = P.E, k = P.k;
-  const uint16_t* lt = P.logits + (size_t)t * E;
-  constexpr int kPer = kMaxExperts / 32;
-  uint32_t key[kPer];
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = (e < E) ? route_key_d(lt[e], e) : 0u;
-  }
-  float mx = 0.f, el[kPer];    // lane (j % 32) keeps exp(l_j - l_max) of choice j in el[j / 32]
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) el[i] = 0.f;
-  for (int j = 0; j < k; ++j) {
-    uint32_t best = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) best = max(best, key[i]);
-    const uint32_t win = __reduce_max_sync(kFull, best);
-#pragma unroll
-    for (int i = 0; i < kPer; ++i)
-      if (key[i] == win) key[i] = 0;                  // keys are unique (the id is in them)
-    const int e = 0xffff - (int)(win & 0xffffu);
-    const uint32_t ord = win >> 16;
-    const float lw = bf16_bits_to_float((ord & 0x8000u) ? (ord & 0x7fffu) : (~ord & 0xffffu));
-    if (j == 0) mx = lw;
-    if ((j & 31) == lane) {
-      s.idx[t * k + j] = e;
-#pragma unroll
-      for (int i = 0; i < kPer; ++i)
-        if ((j >> 5) == i) el[i] = expf(lw - mx);
-      if (slot_of(P.slot, e) >= 0) atomicOr(&s.present[e >> 5], 1u << (e & 31));
-    }
-  }
-  float sum = 0.f;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) sum += el[i];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    const int j = 32 * i + lane;
-    if (j < k) s.wts[t * k + j] = el[i] / sum;
-  }
-}
-
-// Routing (or the given routing), activations into shared memory, active-expert list, and per
-// (active expert, token) router weights. Four CTA barriers, each phase of constant depth.
-__device__ void build_plan(DecSmem& s, const DecParams& P, uint8_t* xs) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int Tk = P.T * P.k, E = P.E;
+// The activations as the K-major bf16 B operand of the gate/up MMAs (all kN rows; rows >= T are
+// left as they are: those MMA columns are never read).
+__device__ void stage_x(const DecParams& P, uint8_t* xs, int tid) {
   const int rowc = P.H / 8;                       // 16-byte chunks per activation row
   const int chunks = P.T * rowc;
-  // activations: issue the loads first so that their latency overlaps the routing
-  constexpr int kPerThr = (kN * 2048 / 8 + kThreads - 1) / kThreads;
-  uint4 xv[kPerThr];
-#pragma unroll
-  for (int i = 0; i < kPerThr; ++i) {
-    const int c = tid + i * kThreads;
-    if (c < chunks) xv[i] = __ldg(reinterpret_cast<const uint4*>(P.x + (size_t)(c / rowc) * P.H) + c % rowc);
-  }
-  if (P.logits) {
-    for (int t = warp; t < P.T; t += kWarps) route_token(s, P, t, lane);
-  } else {
-    for (int p = tid; p < Tk; p += kThreads) {
-      const int e = P.idx_in[p];
-      s.idx[p] = e;
-      s.wts[p] = P.wts_in[p];
-      if ((unsigned)e < (unsigned)E && slot_of(P.slot, e) >= 0) atomicOr(&s.present[e >> 5], 1u << (e & 31));
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kPerThr; ++i) {
-    const int c = tid + i * kThreads;
-    if (c < chunks) *reinterpret_cast<uint4*>(xs + kmajor_off(c / rowc, (c % rowc) * 8)) = xv[i];
-  }
-  for (int c = tid + kPerThr * kThreads; c < chunks; c += kThreads)
+  for (int c = tid; c < chunks; c += kThreads)
     *reinterpret_cast<uint4*>(xs + kmajor_off(c / rowc, (c % rowc) * 8)) =
         __ldg(reinterpret_cast<const uint4*>(P.x + (size_t)(c / rowc) * P.H) + c % rowc);
-  __syncthreads();
-  // active experts in ascending id: rank = set bits below in the presence bitmap
-  if (tid < E) {
-    const int w = tid >> 5;
-    if ((s.present[w] >> (tid & 31)) & 1u) {
-      int a = __popc(s.present[w] & ((1u << (tid & 31)) - 1u));
-      for (int i = 0; i < w; ++i) a += __popc(s.present[i]);
-      s.act[a] = tid;
-      s.aidx[tid] = a;
-    }
-  }
-  if (P.logits && P.idx_out && blockIdx.x == 0)
-    for (int p = tid; p < Tk; p += kThreads) {
-      P.idx_out[p] = s.idx[p];
-      P.wts_out[p] = s.wts[p];
-    }
-  __syncthreads();
-  for (int p = tid; p < Tk; p += kThreads) {
-    const int e = s.idx[p];
-    if ((unsigned)e >= (unsigned)E || !((s.present[e >> 5] >> (e & 31)) & 1u)) continue;
-    const int a = s.aidx[e], t = p / P.k;
-    const uint32_t old = atomicOr(&s.tokmask[a], 1u << t);
-    if ((old >> t) & 1u) s.over = 1;             // a token routed twice to one expert
-    s.wtok[a][t] = s.wts[p];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int n = 0;
-    for (int i = 0; i < (E + 31) / 32; ++i) n += __popc(s.present[i]);
-    s.nact = s.over ? 0 : n;
-    if (s.over) report_status(P.ctl, MOE_ERR_ARG, kSiteOver);
-  }
-  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ DecParams P) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecSmem& s = *reinterpret_cast<DecSmem*>(smem_raw);
   uint8_t* xs = smem_raw + sizeof(DecSmem);
+  uint8_t* ring = xs + (size_t)kN * P.H * 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NS = P.nstages;
 
   // ---- set-up that does not read the previous kernel's results: overlaps it under PDL
   if (warp == 2) {
-    if (lane < kStages) { tc::mbar_init(&s.full[lane], 1); tc::mbar_init(&s.empty[lane], 4); }
-    if (lane < kABufs) { tc::mbar_init(&s.afull[lane], 4); tc::mbar_init(&s.aempty[lane], 1); }
-    if (lane < 2) {
-      tc::mbar_init(&s.gfull[lane], 1); tc::mbar_init(&s.gempty[lane], 4);
-      tc::mbar_init(&s.bfull[lane], 1); tc::mbar_init(&s.bempty[lane], 1);
+    if (lane < kMaxStages) {
+      tc::mbar_init(&s.full[lane], 1);
+      tc::mbar_init(&s.empty[lane], 2 * kDqWarpsPerGroup + kIssuers);   // dequant warps + MMA commits
+      tc::mbar_init(&s.hfull[lane], 1);
+    }
+    if (lane < kABufs) { tc::mbar_init(&s.afull[lane], kDqWarpsPerGroup); tc::mbar_init(&s.aempty[lane], 1); }
+    if (lane < kIssuers * kAcc) {
+      tc::mbar_init(&s.accfull[0][0] + lane, 1);
+      tc::mbar_init(&s.accempty[0][0] + lane, 4);
     }
     if (lane == 0) {
-      tc::mbar_init(&s.hfull, 1);
-      tc::mbar_init(&s.drain, 1);
+      tc::mbar_init(&s.drain[0], 1);
+      tc::mbar_init(&s.drain[1], 1);
       s.abort = 0;
-      s.over = 0;
     }
     tc::fence_barrier_init();
   }
@@ -289,239 +163,342 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     tc::tmem_alloc<kTmemCols>(&s.tmem_base);
     tc::tc_fence_before();
   }
-  for (int i = tid; i < kMaxExperts / 32; i += kThreads) s.present[i] = 0;
-  for (int i = tid; i < kMaxExperts; i += kThreads) s.tokmask[i] = 0;
-  for (int i = tid; i < kMaxExperts * kMaxT; i += kThreads) (&s.wtok[0][0])[i] = 0.f;
-  for (int i = tid; i < (int)(sizeof(s.bdown) / 16); i += kThreads)
-    reinterpret_cast<uint4*>(&s.bdown[0][0])[i] = make_uint4(0, 0, 0, 0);
-  for (int i = tid + P.T * (P.H / 8); i < kN * (P.H / 8); i += kThreads)   // token rows >= T stay zero
-    *reinterpret_cast<uint4*>(xs + kmajor_off(i / (P.H / 8), (i % (P.H / 8)) * 8)) = make_uint4(0, 0, 0, 0);
+  route_clear(s.rs, tid, kThreads);
   __syncthreads();
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) trace_at(P, 0);
-  build_plan(s, P, xs);
+  route_begin(s.rs, P, tid, kThreads);
+  stage_x(P, xs, tid);
+  __syncthreads();
+  route_finish(s.rs, P, tid, kThreads);
   tc::tc_fence_after();
   tc::fence_proxy_async_smem();
   __syncthreads();
-  if (tid == 0) trace_at(P, 1);
+  if (tid == 0) { trace_at(P, 1); trace_clk(P, 7); }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const uint32_t tmem = s.tmem_base;
-  const int IB = P.I / kRowBlock, GH = P.H / kGroup, GI = P.I / kGroup, HB = P.H / kRowBlock;
-  const int NF = P.I / kIF;                                   // units per expert
-  const int U_total = s.nact * NF;
-  const int G = gridDim.x;
-  const int my_units = ((int)blockIdx.x < U_total) ? (U_total - 1 - (int)blockIdx.x) / G + 1 : 0;
+  const int G = gridDim.x, cta = blockIdx.x;
+  Plan pl;
+  pl.init(s.rs.nact, P.H, P.I, G, cta);
   volatile int* abort = &s.abort;
-  const size_t w13_bytes = (size_t)P.I * P.H, s13_count = (size_t)2 * P.I * GH;
-  const size_t w2_bytes = (size_t)P.H * P.I / 2, s2_count = (size_t)P.H * GI;
-  const int stages_per_unit = GH + HB;
+  const int T = P.T;
+  const size_t w13_bytes = (size_t)P.I * P.H, s13_count = (size_t)2 * P.I * pl.nH;
+  const size_t w2_bytes = (size_t)P.H * P.I / 2, s2_count = (size_t)P.H * pl.nI;
+  auto stage_w = [&](int st) { return ring + (size_t)st * kStageBytes; };
+  auto stage_s = [&](int st) { return ring + (size_t)st * kStageBytes + kStageW; };
+  auto stage_h = [&](int st) { return ring + (size_t)st * kStageBytes + kStageW + kStageS; };
+  const int nrg = T > 8 ? 2 : 1;               // 8-token row groups of the h operand
+  const int a_base2 = pl.e1 - pl.b1;           // tile counter of this CTA's first phase-2 tile
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (whole warp)
+    // Lane 0 posts the expected bytes; lanes 0..3 issue the copies of a stage side by side.
     const uint64_t pol = tc::policy_evict_first();
     int it = 0;
-    bool ok = true;
-    for (int n = 0; n < my_units && ok; ++n) {
-      const int u = blockIdx.x + n * G;
-      const int e = s.act[u / NF], sl = slot_of(P.slot, e);
-      const int i0 = (u % NF) * kIF, rb = i0 / kRowBlock, r0 = i0 % kRowBlock;
-      const uint8_t* w13e = P.w13 + (size_t)sl * w13_bytes;
-      const uint16_t* s13e = P.s13 + (size_t)sl * s13_count;
-      const uint8_t* w2e = P.w2 + (size_t)sl * w2_bytes;
-      const uint16_t* s2e = P.s2 + (size_t)sl * s2_count;
-      for (int ti = 0; ti < stages_per_unit; ++ti, ++it) {
-        const int st = it % kStages;
-        if (!warp_wait(&s.empty[st], ((it / kStages) & 1) ^ 1, abort)) { ok = false; break; }
-        if (lane == 0) {
-          if (it == 0) trace_at(P, 2);
-          if (ti < GH) {
-            // rows 0..63: gate rows i0.., rows 64..127: the matching up rows, K group ti
-            const size_t tg = (size_t)rb * GH + ti, tu = (size_t)(IB + rb) * GH + ti;
-            tc::mbar_arrive_expect_tx(&s.full[st], 8192 + 256);
-#pragma unroll
-            for (int kq = 0; kq < 4; ++kq) {
-              tc::bulk_g2s(s.stage[st] + kq * 2048, w13e + tg * kTileBytes + kq * 2048 + r0 * 16, 1024, &s.full[st], pol);
-              tc::bulk_g2s(s.stage[st] + kq * 2048 + 1024, w13e + tu * kTileBytes + kq * 2048 + r0 * 16, 1024,
-                           &s.full[st], pol);
-            }
-            tc::bulk_g2s(&s.scale[st][0], s13e + tg * kRowBlock + r0, 128, &s.full[st], pol);
-            tc::bulk_g2s(&s.scale[st][64], s13e + tu * kRowBlock + r0, 128, &s.full[st], pol);
-          } else {
-            // W2 rows of H-block hb, the unit's 64-wide K half of I-group rb
-            const size_t t2 = (size_t)(ti - GH) * GI + rb;
-            tc::mbar_arrive_expect_tx(&s.full[st], 4096 + 256);
-            tc::bulk_g2s(s.stage[st], w2e + t2 * kTileBytes + (r0 / kIF) * 4096, 4096, &s.full[st], pol);
-            tc::bulk_g2s(&s.scale[st][0], s2e + t2 * kRowBlock, 256, &s.full[st], pol);
+    bool ok = true, h_ready = false;
+    int first2 = -1;                         // stage index of the first phase-2 stage
+    int pend_n = 0, pend_st[kMaxStages], pend_u[kMaxStages], pend_len[kMaxStages];
+    int h_issued[kMaxStages];                // h copies issued per slot (for the final drain)
+    for (int i = 0; i < kMaxStages; ++i) h_issued[i] = 0;
+    const int h_target = pl.m * pl.nI;
+    auto issue_h = [&](int st, int u, int n) {
+      const int j = (u % pl.tpr2) / pl.nI, g0 = u % pl.nI;
+      if (lane == 0) tc::mbar_arrive_expect_tx(&s.hfull[st], (uint32_t)(n * kHTile * nrg));
+      __syncwarp();
+      if (lane < nrg)
+        tc::bulk_g2s(stage_h(st) + lane * (kTilesPerStage * kHTile),
+                     P.hbuf + ((size_t)(j * 2 + lane) * pl.nI + g0) * kHTile, (uint32_t)(n * kHTile), &s.hfull[st], pol);
+      ++h_issued[st];
+    };
+    auto poll_h = [&]() -> bool {            // warp-uniform
+      int v = 0;
+      if (lane == 0) v = tc::ld_acquire(P.hdone) >= h_target;
+      return __shfl_sync(kFull, v, 0) != 0;
+    };
+    auto wait_h = [&]() -> bool {            // every feature block's h is in global memory
+      int okw = 1;
+      if (lane == 0) {
+        const long long t0 = clock64();
+        while (tc::ld_acquire(P.hdone) < h_target) {
+          if (*abort || clock64() - t0 > tc::kWaitTimeoutCycles) {
+            trace_val(P, 8, tc::ld_acquire(P.hdone));
+            trace_val(P, 9, h_target);
+            okw = 0;
+            break;
           }
+          __nanosleep(64);
         }
       }
-    }
-    if (!ok && lane == 0) report_abort(s, P, kSiteStage);
-    if (lane == 0) trace_at(P, 3);
-    if (lane == 0) {   // no bulk copy may still be landing in shared memory when the CTA leaves
-      const int nw = it < kStages ? it : kStages;
-      for (int i = 0; i < nw; ++i) {
-        const int j = it - 1 - i;
-        volatile int never = 0;
-        tc::mbar_wait(&s.full[j % kStages], (j / kStages) & 1, &never);
+      return __shfl_sync(kFull, okw, 0) != 0;
+    };
+    auto flush_h = [&]() -> bool {
+      if (!h_ready) {
+        if (!wait_h()) return false;
+        fence_proxy_async_global();
+        h_ready = true;
+        if (lane == 0) trace_at(P, 4);
+      }
+      for (int i = 0; i < pend_n; ++i) issue_h(pend_st[i], pend_u[i], pend_len[i]);
+      pend_n = 0;
+      return true;
+    };
+    for (int phase = 1; phase <= 2 && ok; ++phase) {
+      const int ub = phase == 1 ? pl.b1 : pl.b2, ue = phase == 1 ? pl.e1 : pl.e2;
+      if (phase == 2 && ub < ue) first2 = it;
+      for (int u = ub; u < ue; ++it) {
+        const int n = phase == 1 ? pl.run1(u) : pl.run2(u);
+        const int st = it % NS;
+        // the slot about to be reused may hold a phase-2 stage still waiting for its h
+        if (!h_ready && first2 >= 0 && it >= NS && it - NS >= first2 && !flush_h()) { ok = false; break; }
+        if (!warp_wait(&s.empty[st], ((it / NS) & 1) ^ 1, abort)) { ok = false; break; }
+        int j, lt;
+        pl.locate(phase, u, j, lt);
+        const int sl = slot_of(P.slot, s.rs.act[j]);
+        const uint8_t* wsrc = phase == 1 ? P.w13 + (size_t)sl * w13_bytes : P.w2 + (size_t)sl * w2_bytes;
+        const uint16_t* ssrc = phase == 1 ? P.s13 + (size_t)sl * s13_count : P.s2 + (size_t)sl * s2_count;
+        if (lane == 0) tc::mbar_arrive_expect_tx(&s.full[st], (uint32_t)(n * (kTileBytes + kRowBlock * 2)));
+        __syncwarp();
+        if (lane == 0) tc::bulk_g2s(stage_w(st), wsrc + (size_t)lt * kTileBytes, (uint32_t)(n * kTileBytes), &s.full[st], pol);
+        if (lane == 1) tc::bulk_g2s(stage_s(st), ssrc + (size_t)lt * kRowBlock, (uint32_t)(n * kRowBlock * 2), &s.full[st], pol);
+        if (lane == 0 && it < 4) trace_clk(P, 12 + it);
+        if (phase == 2) {
+          if (!h_ready && poll_h()) {
+            fence_proxy_async_global();
+            h_ready = true;
+            if (lane == 0) trace_at(P, 4);
+          }
+          if (h_ready) {
+            if (!flush_h()) { ok = false; ++it; break; }
+            issue_h(st, u, n);
+          } else {
+            pend_st[pend_n] = st; pend_u[pend_n] = u; pend_len[pend_n] = n; ++pend_n;
+          }
+        }
+        u += n;
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) trace_at(P, 3);
+    if (ok && pend_n > 0 && !flush_h()) ok = false;
+    if (!ok && lane == 0) report_abort(s, P, kSiteHDone);
+    // no bulk copy may still be landing in shared memory when the CTA leaves
+    if (lane == 0) {
+      volatile int never = 0;
+      const int nw = it < NS ? it : NS;
+      for (int i = 0; i < nw; ++i) {
+        const int jst = it - 1 - i;
+        tc::mbar_wait(&s.full[jst % NS], (jst / NS) & 1, &never);
+      }
+      for (int st = 0; st < NS; ++st)
+        if (h_issued[st] > 0) tc::mbar_wait(&s.hfull[st], (h_issued[st] - 1) & 1, &never);
+    }
+    __syncwarp();
+  } else if (warp == kIssuerWarp0 || warp == kIssuerWarp1) {
+    // ------------------------------------------------------------ MMA issuers
+    // issuer `me` takes the tiles whose running index has parity `me` and accumulates them into
+    // its own accumulators; the epilogue adds the two partial sums of each block.
+    const int me = warp == kIssuerWarp0 ? 0 : 1;
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_bf16_f32(128, kN);
       const uint32_t xbase = tc::smem_u32(xs);
-      constexpr uint32_t lbo = (kN / 8) * 128;
-      int a_it = 0;
-      bool ok = true;
-      for (int n = 0; n < my_units && ok; ++n) {
-        const int db = n & 1;
-        if (!tc::mbar_wait(&s.gempty[db], ((n >> 1) & 1) ^ 1, abort)) { ok = false; report_abort(s, P, kSiteD); break; }
-        tc::tc_fence_after();
-        for (int g = 0; g < GH && ok; ++g, ++a_it) {
-          const int ab = a_it % kABufs;
-          if (!tc::mbar_wait(&s.afull[ab], (a_it / kABufs) & 1, abort)) { ok = false; report_abort(s, P, kSiteABuf); break; }
-          tc::tc_fence_after();
-          const uint32_t a = tmem + kAColBase + ab * 64;
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bdesc = tc::smem_desc(xbase + ((g * kGroup + kk * 16) / 8) * lbo, lbo, 128, 0);
-            tc::mma_ts(tmem + kDguCol + db * kN, a + kk * 8, bdesc, idesc, (g > 0 || kk > 0) ? 1u : 0u);
+      int it = 0, a_it = 0, sg = 0;
+      uint32_t hphase = 0;                      // bit st: parity of the next hfull[st] completion
+      bool ok = true, started = false;
+      for (int phase = 1; phase <= 2 && ok; ++phase) {
+        const int ub = phase == 1 ? pl.b1 : pl.b2, ue = phase == 1 ? pl.e1 : pl.e2;
+        const int per = phase == 1 ? pl.nH : pl.tpr2;
+        for (int u = ub; u < ue && ok; ++it) {
+          const int n = phase == 1 ? pl.run1(u) : pl.run2(u);
+          const int st = it % NS;
+          uint32_t hb = 0;
+          if (phase == 2) {
+            if (!tc::mbar_wait(&s.hfull[st], (hphase >> st) & 1, abort)) { ok = false; report_abort(s, P, kSiteH); break; }
+            hphase ^= 1u << st;
+            tc::tc_fence_after();
+            hb = tc::smem_u32(stage_h(st));
           }
-          tc::mma_commit(&s.aempty[ab]);
-        }
-        if (!ok) break;
-        tc::mma_commit(&s.gfull[db]);
-        const int bb = n & 1;
-        if (!tc::mbar_wait(&s.bfull[bb], (n >> 1) & 1, abort)) { ok = false; report_abort(s, P, kSiteB); break; }
-        tc::tc_fence_after();
-        const uint32_t hbase = tc::smem_u32(s.bdown[bb]);
-        for (int hb = 0; hb < HB && ok; ++hb, ++a_it) {
-          const int ab = a_it % kABufs;
-          if (!tc::mbar_wait(&s.afull[ab], (a_it / kABufs) & 1, abort)) { ok = false; report_abort(s, P, kSiteABuf); break; }
-          tc::tc_fence_after();
-          const uint32_t a = tmem + kAColBase + ab * 64;
+          for (int i = 0; i < n; ++i, ++a_it) {
+            const int uu = u + i;
+            const bool seg_first = uu == ub || uu % per == 0;
+            const bool seg_last = uu == ue - 1 || (uu + 1) % per == 0;
+            const int ac = sg % kAcc;
+            if (seg_first) {
+              started = false;
+              if (!tc::mbar_wait(&s.accempty[me][ac], ((sg / kAcc) & 1) ^ 1, abort)) { ok = false; report_abort(s, P, kSiteAcc); break; }
+              tc::tc_fence_after();
+            }
+            if ((a_it & 1) == me) {
+              const int ab = a_it % kABufs;
+              if (!tc::mbar_wait(&s.afull[ab], (a_it / kABufs) & 1, abort)) { ok = false; report_abort(s, P, kSiteABuf); break; }
+              tc::tc_fence_after();
+              if (a_it < 8) trace_clk(P, 40 + a_it);
+              const uint32_t a = tmem + kAColBase + ab * 64, d = tmem + kAccCol + (me * kAcc + ac) * kN;
+              if (phase == 1) {
+                const int g = uu % pl.nH;
 #pragma unroll
-          for (int kk = 0; kk < kIF / 16; ++kk) {
-            const uint64_t bdesc = tc::smem_desc(hbase + kk * 2 * lbo, lbo, 128, 0);
-            tc::mma_ts(tmem + kDhCol + hb * kN, a + kk * 8, bdesc, idesc, (n > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint64_t bdesc = tc::smem_desc(xbase + (uint32_t)((g * kGroup + kk * 16) / 8) * 256u, 256, 128, 0);
+                  tc::mma_ts(d, a + kk * 8, bdesc, idesc, (started || kk > 0) ? 1u : 0u);
+                }
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint64_t bdesc = tc::smem_desc(hb + (uint32_t)(i * kHTile + kk * 256), 128,
+                                                       kTilesPerStage * kHTile, 0);
+                  tc::mma_ts(d, a + kk * 8, bdesc, idesc, (started || kk > 0) ? 1u : 0u);
+                }
+              }
+              started = true;
+              tc::mma_commit(&s.aempty[ab]);
+              if (a_it < 8) trace_clk(P, 48 + a_it);
+            }
+            if (seg_last) {
+              tc::mma_commit(&s.accfull[me][ac]);
+              ++sg;
+            }
           }
-          tc::mma_commit(&s.aempty[ab]);
+          if (!ok) break;
+          tc::mma_commit(&s.empty[st]);     // the stage's h operand is no longer read by this issuer
+          u += n;
         }
-        tc::mma_commit(&s.bempty[bb]);
       }
-      if (ok && my_units > 0) tc::mma_commit(&s.hfull);
-      tc::mma_commit(&s.drain);
+      tc::mma_commit(&s.drain[me]);
       volatile int never = 0;
-      if (!tc::mbar_wait(&s.drain, 0, &never)) report_status(P.ctl, MOE_ERR_TIMEOUT, kSiteDrain);
+      if (!tc::mbar_wait(&s.drain[me], 0, &never)) report_status(P.ctl, MOE_ERR_TIMEOUT, kSiteDrain);
     }
     __syncwarp();
-  } else if (warp >= kDqWarp0) {
+  } else if (warp >= kDqWarp0 && warp < kDqWarp0 + 2 * kDqWarpsPerGroup) {
     // ------------------------------------------------------------ dequantisers -> TMEM
-    // two groups of four warps take alternate stages; a thread owns row r of the stage
-    const int quarter = warp & 3, grp = (warp - kDqWarp0) >> 2;
+    // two groups of four warps take alternate tiles (group = parity of the running tile index),
+    // a thread owns one row of its group's tiles; every stage barrier is waited for in order
+    const int quarter = warp & 3, grp = (warp - kDqWarp0) / kDqWarpsPerGroup;
     const int r = quarter * 32 + lane;
     const uint32_t taddr_row = tmem + ((uint32_t)(quarter * 32) << 16) + kAColBase;
     const __nv_bfloat162 off136 = __floats2bfloat162_rn(136.f, 136.f);
-    int it = 0;
+    int it = 0, a_it = 0;
     bool ok = true;
-    for (int n = 0; n < my_units && ok; ++n) {
-      for (int ti = 0; ti < stages_per_unit; ++ti, ++it) {
-        if ((it & 1) != grp) continue;
-        const int st = it % kStages;
-        const int halves = (ti < GH) ? 2 : 1;       // 128 K (gate/up) or 64 K (down) per row
-        if (!warp_wait(&s.full[st], (it / kStages) & 1, abort)) { ok = false; break; }
-        uint4 c[4];
+    for (int phase = 1; phase <= 2 && ok; ++phase) {
+      const int ub = phase == 1 ? pl.b1 : pl.b2, ue = phase == 1 ? pl.e1 : pl.e2;
+      for (int u = ub; u < ue && ok; ++it) {
+        const int n = phase == 1 ? pl.run1(u) : pl.run2(u);
+        u += n;
+        const int st = it % NS;
+        if (!warp_wait(&s.full[st], (it / NS) & 1, abort)) { ok = false; break; }
+        const uint8_t* sw = stage_w(st) + r * 16;
+        const uint16_t* ss = reinterpret_cast<const uint16_t*>(stage_s(st));
+        // my tiles in this stage: i = first, first + 2, ...; the stage is released after the
+        // loads of the last of them (or at once when there is none)
+        const int first = (a_it & 1) == grp ? 0 : 1;
+        const int last = (first < n) ? first + ((n - 1 - first) & ~1) : -1;
+        if (last < 0) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&s.empty[st]);
+        }
+        for (int i = first; i < n; i += 2) {
+          const int ai = a_it + i;
+          uint4 c[4];
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq)
-          c[kq] = (kq < 2 * halves) ? *reinterpret_cast<const uint4*>(s.stage[st] + kq * 2048 + r * 16)
-                                    : make_uint4(0, 0, 0, 0);
-        const uint32_t sb = s.scale[st][r];
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&s.empty[st]);
-        const uint32_t s2u = sb | (sb << 16);
-        const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
-        const int ab = it % kABufs;
-        if (!warp_wait(&s.aempty[ab], ((it / kABufs) & 1) ^ 1, abort)) { ok = false; break; }
-        tc::tc_fence_after();
-        dequant_half(c[0], c[1], s2, off136, taddr_row + ab * 64);
-        if (halves == 2) dequant_half(c[2], c[3], s2, off136, taddr_row + ab * 64 + 32);
-        tc::tmem_wait_st();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&s.afull[ab]);
+          for (int kq = 0; kq < 4; ++kq) c[kq] = *reinterpret_cast<const uint4*>(sw + i * kTileBytes + kq * 2048);
+          const uint32_t sb = ss[i * kRowBlock + r];
+          if (i == last) {
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&s.empty[st]);
+          }
+          const uint32_t s2u = sb | (sb << 16);
+          const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+          const int ab = ai % kABufs;
+          if (!warp_wait(&s.aempty[ab], ((ai / kABufs) & 1) ^ 1, abort)) { ok = false; break; }
+          tc::tc_fence_after();
+          if (quarter == 0 && lane == 0 && ai < 8) trace_clk(P, 24 + ai);
+          dequant_half(c[0], c[1], s2, off136, taddr_row + ab * 64);
+          dequant_half(c[2], c[3], s2, off136, taddr_row + ab * 64 + 32);
+          tc::tmem_wait_st();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&s.afull[ab]);
+          if (quarter == 0 && lane == 0 && ai < 8) trace_clk(P, 32 + ai);
+        }
+        a_it += n;
       }
     }
-  } else {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogues (warps 2..5)
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;          // rows 0..63: gate of feature r, 64..127: up of r-64
-    const int etid = tid - kEpiWarp0 * 32;      // 0..127 (warp 2 holds rows 64..95)
+    const int r = quarter * 32 + lane;          // accumulator row (TMEM lane)
+    const int etid = tid - kEpiWarp0 * 32;      // 0..127
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
-    // Every exit decision is taken after the second named barrier from the CTA's abort flag,
-    // so the four warps always meet at the same barriers (a failed wait raises the flag).
-    for (int n = 0; n < my_units; ++n) {
-      const int u = blockIdx.x + n * G;
-      const int a = u / NF;
-      const int db = n & 1;
-      const bool g_ok = warp_wait(&s.gfull[db], (n >> 1) & 1, abort);
-      uint32_t v[kN];
+    const int nI = pl.nI;
+    int sg = 0;
+    bool stop = false;
+    // Each decision is taken by one thread between two named barriers and read by all, so the
+    // four warps always meet at the same barriers.
+    for (int phase = 1; phase <= 2 && !stop; ++phase) {
+      const int ub = phase == 1 ? pl.b1 : pl.b2, ue = phase == 1 ? pl.e1 : pl.e2;
+      if (ub >= ue) continue;
+      const int per = phase == 1 ? pl.nH : pl.tpr2;
+      const int a0 = phase == 1 ? 0 : a_base2;
+      for (int key = ub / per; key <= (ue - 1) / per; ++key, ++sg) {
+        const int ac = sg % kAcc;
+        // tiles of this block in the CTA's running tile index; which issuers had some
+        const int t0 = max(ub, key * per), t1 = min(ue, (key + 1) * per);
+        const int af = a0 + (t0 - ub);
+        const bool has0 = (t1 - t0) >= 2 || (af & 1) == 0, has1 = (t1 - t0) >= 2 || (af & 1) == 1;
+        bool ok = warp_wait(&s.accfull[0][ac], (sg / kAcc) & 1, abort);
+        ok = ok && warp_wait(&s.accfull[1][ac], (sg / kAcc) & 1, abort);
+        if (etid == 0 && sg < 8) trace_clk(P, 56 + sg);
+        float* part = (phase == 1 ? P.p1 : P.p2) + (size_t)(key + cta) * T * kRowBlock;
+        if (ok) {
+          tc::tc_fence_after();
+          uint32_t v0[kN], v1[kN];
+          tc::tmem_ld16(trow + kAccCol + ac * kN, v0);
+          tc::tmem_ld16(trow + kAccCol + (kAcc + ac) * kN, v1);
+          tc::tmem_wait_ld();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            tc::mbar_arrive(&s.accempty[0][ac]);
+            tc::mbar_arrive(&s.accempty[1][ac]);
+          }
 #pragma unroll
-      for (int t = 0; t < kN; ++t) v[t] = 0;
-      if (g_ok) {
-        tc::tc_fence_after();
-        tc::tmem_ld16(trow + kDguCol + db * kN, v);
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&s.gempty[db]);
-        if (r < kIF) {
-#pragma unroll
-          for (int t = 0; t < kN; ++t) s.gx[r][t] = __uint_as_float(v[t]);
+          for (int t = 0; t < kN; ++t)
+            if (t < T)
+              part[t * kRowBlock + r] = (has0 ? __uint_as_float(v0[t]) : 0.f) + (has1 ? __uint_as_float(v1[t]) : 0.f);
+          __threadfence();
         }
-      }
-      tc::named_bar_sync(1, 128);
-      if (r >= kIF && g_ok && !*abort) {
-        const int bb = n & 1;
-        if (warp_wait(&s.bempty[bb], ((n >> 1) & 1) ^ 1, abort)) {
-          const int f = r - kIF;
-          const uint32_t tm = s.tokmask[a];
-          uint8_t* dst = s.bdown[bb];
+        tc::named_bar_sync(1, 128);
+        if (etid == 0) s.epi_dec = *abort ? -1 : (block_arrive(pl, P, phase, key) ? 1 : 0);
+        tc::named_bar_sync(1, 128);
+        const int d = s.epi_dec;
+        if (etid == 0) trace_val(P, 10, sg + 1);
+        if (d < 0) { stop = true; break; }
+        if (d == 1 && phase == 1) {
+          // h = w * silu(gate) * up for feature block fb of selected expert j, as bf16 h tiles
+          const int j = key / (2 * nI), fb = (key % (2 * nI)) % nI;
+          if (etid < T) s.wsel[etid] = route_weight(s.rs, P, etid, s.rs.act[j]);
+          tc::named_bar_sync(1, 128);
+          float g[kN], up[kN];
+          gate_up_sums<kN>(pl, P, j, fb, etid, g, up);
 #pragma unroll
           for (int t = 0; t < kN; ++t) {
-            float hv = 0.f;
-            if ((tm >> t) & 1u) {
-              const float g = s.gx[f][t];
-              hv = g / (1.f + expf(-g)) * __uint_as_float(v[t]) * s.wtok[a][t];
+            if (t < T) {
+              const float w = s.wsel[t];
+              const float hv = (w != 0.f) ? swiglu(g[t], up[t]) * w : 0.f;
+              uint8_t* dst = P.hbuf + ((size_t)(j * 2 + (t >> 3)) * nI + fb) * kHTile;
+              *reinterpret_cast<__nv_bfloat16*>(dst + (etid >> 3) * 128 + (t & 7) * 16 + (etid & 7) * 2) =
+                  __float2bfloat16_rn(hv);
             }
-            *reinterpret_cast<__nv_bfloat16*>(dst + kmajor_off(t, f)) = __float2bfloat16_rn(hv);
           }
-          tc::fence_proxy_async_smem();
+          fence_proxy_async_global();
+          __threadfence();
+          tc::named_bar_sync(1, 128);
+          if (etid == 0) tc::red_release_add(P.hdone, 1);
+        } else if (d == 1) {
+          output_block<kN>(pl, P, key, etid);
         }
       }
-      tc::named_bar_sync(1, 128);
-      if (*abort) break;
-      if (etid == 0) tc::mbar_arrive(&s.bfull[n & 1]);
     }
-    const bool ok = !*abort;
-    // the CTA's partial output: rows hb*128 + r, all tokens
-    float* yp = P.ypart + (size_t)blockIdx.x * P.T * P.H;
-    if (my_units > 0 && ok && warp_wait(&s.hfull, 0, abort)) {
-      tc::tc_fence_after();
-      for (int hb = 0; hb < HB; ++hb) {
-        uint32_t y[kN];
-        tc::tmem_ld16(trow + kDhCol + hb * kN, y);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int t = 0; t < kN; ++t)
-          if (t < P.T) yp[(size_t)t * P.H + hb * kRowBlock + r] = __uint_as_float(y[t]);
-      }
-    } else {
-      for (int i = etid; i < P.T * P.H; i += 128) yp[i] = 0.f;
-    }
-    if (etid == 0) trace_at(P, 4);
+    if (etid == 0) trace_at(P, 5);
   }
 
   tc::tc_fence_before();
@@ -530,109 +507,27 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     tc::tc_fence_after();
     tc::tmem_dealloc<kTmemCols>(tmem);
   }
-
-  // ---- grid-wide barrier (every CTA is resident: one CTA per SM, grid <= SM count)
-  if (tid == 0) {
-    const int gen = tc::ld_acquire(P.ctl + kCtlBarGen);
-    __threadfence();
-    if (atomicAdd(P.ctl + kCtlBarCount, 1) == G - 1) {
-      P.ctl[kCtlBarCount] = 0;
-      tc::red_release_add(P.ctl + kCtlBarGen, 1);
-    } else {
-      const long long t0 = clock64();
-      while (tc::ld_acquire(P.ctl + kCtlBarGen) == gen) {
-        if (clock64() - t0 > tc::kWaitTimeoutCycles) {
-          report_status(P.ctl, MOE_ERR_TIMEOUT, kSiteGrid);
-          break;
-        }
-        __nanosleep(64);
-      }
-    }
-    trace_at(P, 5);
-  }
-  __syncthreads();
-
-  // ---- final reduction: this CTA's slice of the T x H outputs, partials summed in CTA order
-  const int total = P.T * P.H;
-  const int per = (total + G - 1) / G;
-  const int e0 = (int)blockIdx.x * per;
-  const int cnt = max(0, min(per, total - e0));
-  if (cnt > 0) {
-    const int stripes = max(1, min(G, kThreads / cnt));
-    const int el = tid % cnt, sp = tid / cnt;
-    float v = 0.f;
-    if (sp < stripes && tid < stripes * cnt)
-      for (int c = sp; c < G; c += stripes) v += __ldcg(P.ypart + (size_t)c * total + e0 + el);
-    s.red[tid] = v;
-    __syncthreads();
-    for (int i = tid; i < cnt; i += kThreads) {
-      float accv = P.accumulate ? __ldcg(P.acc + e0 + i) : 0.f;
-      for (int q = 0; q < stripes; ++q) accv += s.red[q * cnt + i];
-      if (P.out) {
-        P.out[e0 + i] = __bfloat16_as_ushort(__float2bfloat16_rn(accv));
-        if (P.accumulate) P.acc[e0 + i] = 0.f;
-      } else {
-        P.acc[e0 + i] = accv;
-      }
-    }
-  }
-  if (tid == 0) trace_at(P, 6);
+  finish_launch(pl, P, abort, tid, kThreads);
 }
 
-int g_num_sms = 0;
-unsigned long long* g_trace = nullptr;
-
-int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
-  return g_num_sms;
+size_t fixed_smem_bytes(int H) { return sizeof(DecSmem) + (size_t)kN * H * 2; }
+int decode_stages(int H) {
+  const long avail = (long)kSmemLimit - (long)fixed_smem_bytes(H);
+  return (int)std::min<long>(kMaxStages, avail > 0 ? avail / kStageBytes : 0);
 }
+size_t decode_smem_bytes(int H) { return fixed_smem_bytes(H) + (size_t)decode_stages(H) * kStageBytes; }
 
-size_t decode_smem_bytes(int H) { return sizeof(DecSmem) + (size_t)kN * H * 2; }
+// h bytes per (selected expert, K group of I): the larger of the two kernels' layouts
+size_t hbuf_per_tile(int T) { return std::max<size_t>(2 * kHTile, gemv_hbuf_per_tile(std::min(T, kGemvMaxT))); }
 
-}  // namespace
-
-// Diagnostics: when set, the fused decode kernel records per-CTA timestamps (64 x u64 per CTA)
-// into this device buffer; NULL turns it off.
-MOE_API void moe_debug_set_decode_trace(void* dev_buffer) {
-  g_trace = static_cast<unsigned long long*>(dev_buffer);
-}
-
-bool ffn_decode_supported(const FfnArgs& a) {
-  return a.T >= 1 && a.T <= kMaxT && a.T * a.k <= kMaxTk && a.E <= kMaxExperts && a.H % kRowBlock == 0 &&
-         a.I % kRowBlock == 0 && a.H / kRowBlock <= kMaxHB && decode_smem_bytes(a.H) <= 227 * 1024;
-}
-
-size_t decode_scratch_bytes(int T, int H, int I, int E, int k) {
-  (void)I; (void)E; (void)k;
-  if (T < 1 || T > kMaxT) return 0;
-  return align_up(sizeof(float) * (size_t)kMaxGrid * T * H, 256);     // per-CTA partial outputs
-}
-
-int ffn_decode(const FfnArgs& a, cudaStream_t s) {
-  const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
-  DecParams P{};
-  P.x = a.x; P.logits = a.logits; P.idx_in = a.idx; P.wts_in = a.wts;
-  P.T = a.T; P.H = a.H; P.I = a.I; P.E = a.E; P.k = a.k;
-  P.w13 = a.w13; P.s13 = a.s13; P.w2 = a.w2; P.s2 = a.s2; P.slot = a.slot;
-  P.idx_out = a.idx_out; P.wts_out = a.wts_out;
-  P.out = a.out; P.acc = reinterpret_cast<float*>(a.ws + L.acc); P.accumulate = a.accumulate ? 1 : 0;
-  P.ctl = reinterpret_cast<int*>(a.ws + L.status);
-  P.ypart = reinterpret_cast<float*>(a.ws + L.dec);
-  P.trace = g_trace;
-  if (!a.logits && (!a.idx || !a.wts)) return fail(MOE_ERR_ARG, "fused decode: routing missing");
-
-  const int max_units = std::min(a.E, a.T * a.k) * (a.I / kIF);
-  const int grid = std::max(1, std::min(std::min(num_sms(), kMaxGrid), max_units));
-  const size_t smem = decode_smem_bytes(a.H);
+int launch_tensor(const DecParams& P0, int grid, cudaStream_t s) {
+  DecParams P = P0;
+  P.nstages = decode_stages(P.H);
+  const size_t smem = decode_smem_bytes(P.H);
   static bool attr_done = false;
   if (!attr_done) {
     if (int rc = check_cuda(cudaFuncSetAttribute(moe_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 227 * 1024), "fused decode: smem attribute"))
+                                                 kSmemLimit), "fused decode: smem attribute"))
       return rc;
     attr_done = true;
   }
@@ -649,6 +544,56 @@ int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   cudaError_t e = cudaLaunchKernelEx(&cfg, moe_decode_kernel, P);
   note_launch();
   return check_cuda(e, "moe_decode_kernel launch");
+}
+
+}  // namespace
+}  // namespace dec
+
+// Diagnostics: when set, the fused decode kernels record per-CTA diagnostics (64 x u64 per CTA)
+// into this device buffer; NULL turns it off.
+MOE_API void moe_debug_set_decode_trace(void* dev_buffer) {
+  dec::g_trace = static_cast<unsigned long long*>(dev_buffer);
+}
+
+bool ffn_decode_supported(const FfnArgs& a) {
+  if (!(a.T >= 1 && a.T <= dec::kMaxT && a.T * a.k <= dec::kMaxTk && a.E <= kMaxExperts && a.H % kRowBlock == 0 &&
+        a.I % kRowBlock == 0 && a.H > 0 && a.I > 0))
+    return false;
+  if (!dec::split_fits(a.T, a.H, a.I, a.E, a.k, dec::kMaxGrid)) return false;
+  return a.T <= dec::kGemvMaxT ? dec::gemv_stages(a.T, a.H) >= 2 : dec::decode_stages(a.H) >= 2;
+}
+
+size_t decode_scratch_bytes(int T, int H, int I, int E, int k) {
+  if (T < 1 || T > dec::kMaxT || H % kRowBlock || I % kRowBlock || E < 1 || k < 1) return 0;
+  return dec::dec_scratch(T, H, I, E, k, dec::hbuf_per_tile(T)).total;
+}
+
+// Batches of up to four tokens run on the CUDA-core kernel, larger ones on the tensor-core one.
+int ffn_decode(const FfnArgs& a, cudaStream_t s) {
+  const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
+  const dec::DecScratch D = dec::dec_scratch(a.T, a.H, a.I, a.E, a.k, dec::hbuf_per_tile(a.T));
+  char* d = a.ws + L.dec;
+  dec::DecParams P{};
+  P.x = a.x; P.logits = a.logits; P.idx_in = a.idx; P.wts_in = a.wts;
+  P.T = a.T; P.H = a.H; P.I = a.I; P.E = a.E; P.k = a.k;
+  P.w13 = a.w13; P.s13 = a.s13; P.w2 = a.w2; P.s2 = a.s2; P.slot = a.slot;
+  P.idx_out = a.idx_out; P.wts_out = a.wts_out;
+  P.out = a.out; P.acc = reinterpret_cast<float*>(a.ws + L.acc); P.accumulate = a.accumulate ? 1 : 0;
+  P.ctl = reinterpret_cast<int*>(a.ws + L.status);
+  P.hcnt = reinterpret_cast<int*>(d + D.hcnt);
+  P.fcnt = reinterpret_cast<int*>(d + D.fcnt);
+  P.hdone = reinterpret_cast<int*>(d + D.hdone);
+  P.p1 = reinterpret_cast<float*>(d + D.p1);
+  P.p2 = reinterpret_cast<float*>(d + D.p2);
+  P.hbuf = reinterpret_cast<uint8_t*>(d + D.hbuf);
+  P.mul16 = 65536u;
+  P.trace = dec::g_trace;
+  if (!a.logits && (!a.idx || !a.wts)) return fail(MOE_ERR_ARG, "fused decode: routing missing");
+
+  const int m_max = std::min(a.E, a.T * a.k);
+  const long tiles1 = (long)m_max * 2 * (a.I / kRowBlock) * (a.H / kGroup);
+  const int grid = (int)std::max<long>(1, std::min<long>(std::min(dec::num_sms(), dec::kMaxGrid), tiles1));
+  return a.T <= dec::kGemvMaxT ? dec::launch_decode_gemv(P, grid, s) : dec::launch_tensor(P, grid, s);
 }
 
 }  // namespace moe
