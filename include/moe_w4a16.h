@@ -159,6 +159,30 @@ int moe_w4a16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16,
                     void* workspace, size_t workspace_bytes,
                     uint16_t* out_bf16, int flags, moe_stream_t stream);
 
+/* moe_w4a16_layer without a caller workspace (the pages have no counterpart: this is a library
+ * convenience). For callers that cannot allocate device memory - a program linking this C
+ * library directly under a device-memory budget fixed up front, or a hot loop where an
+ * allocation would synchronise the device - the workspace is a fixed 16 MiB array that the
+ * library keeps in device memory (enough for the fused decode path at up to 16 tokens on a
+ * 2048-wide, 64-expert, top-8 layer). Arguments as moe_w4a16_layer, minus the workspace.
+ *  - The first call on a device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture on the device.
+ *  - Every call on a device shares the array: calls that can run at the same time (other
+ *    streams, other host threads) race, so the caller must serialise them.
+ *  - Each call clears, on `stream`, the parts that must start at zero (status/control block
+ *    and the fused-decode counters). Device-side failures are not reported by this entry.
+ *  - Nothing is allocated.
+ * Errors: MOE_ERR_SHAPE when these sizes need more than the array holds (use moe_w4a16_layer
+ * with a caller workspace), MOE_ERR_ARG for MOE_FLAG_ACCUMULATE (the fp32 accumulator would be
+ * shared by every call) and the errors of moe_w4a16_layer. */
+int moe_w4a16_layer_noalloc(const uint16_t* x_bf16, const uint16_t* logits_bf16,
+                            int T, int H, int I, int E, int k,
+                            const uint8_t* w13, const uint16_t* s13,
+                            const uint8_t* w2, const uint16_t* s2,
+                            const int32_t* slot_of_expert,
+                            int32_t* idx, float* wts,
+                            uint16_t* out_bf16, int flags, moe_stream_t stream);
+
 /* ---- GPU slot cache (abstract: "configurable GPU-resident slot cache", experts kept in
  * pinned host memory). One cache per layer: S device slots, each holding one expert's packed
  * W13, W2 and their scales; misses are copied from the pinned host bank with

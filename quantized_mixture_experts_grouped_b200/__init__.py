@@ -54,6 +54,7 @@ def _load() -> ctypes.CDLL:
         "moe_workspace_status": ([P, P, c.POINTER(I)], I),
         "moe_w4a16_ffn": ([P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P, I, P], I),
         "moe_w4a16_layer": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P, I, P], I),
+        "moe_w4a16_layer_noalloc": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, I, P], I),
         "moe_slot_cache_create": ([I, I, I, I, P, P, P, P, P, P, P, P, c.POINTER(P)], I),
         "moe_slot_cache_destroy": ([P], None),
         "moe_slot_cache_fail_copy_after": ([P, I], None),
@@ -155,6 +156,14 @@ def moe_w4a16_layer(x, logits, k: int, w13, s13, w2, s2, H: int, I: int, idx, wt
     _err(lib.moe_w4a16_layer(_p(x), _p(logits), T, H, I, E, k, _p(w13), _p(s13), _p(w2), _p(s2),
                              _p(slot_of_expert), _p(idx), _p(wts), _p(ws), ws.numel() * ws.element_size(),
                              _p(out), flags, _s(stream)))
+
+
+def moe_w4a16_layer_noalloc(x, logits, k: int, w13, s13, w2, s2, H: int, I: int, idx, wts, out,
+                            slot_of_expert=None, flags: int = MOE_PATH_AUTO, stream=None):
+    """moe_w4a16_layer with the library's static device scratch as its workspace (no allocation)."""
+    T, E = logits.shape
+    _err(lib.moe_w4a16_layer_noalloc(_p(x), _p(logits), T, H, I, E, k, _p(w13), _p(s13), _p(w2), _p(s2),
+                                     _p(slot_of_expert), _p(idx), _p(wts), _p(out), flags, _s(stream)))
 
 
 class SlotCache:

@@ -568,6 +568,12 @@ size_t decode_scratch_bytes(int T, int H, int I, int E, int k) {
   return dec::dec_scratch(T, H, I, E, k, dec::hbuf_per_tile(T)).total;
 }
 
+// Bytes at the start of the fused-decode scratch that hold counters (zero between launches).
+size_t decode_counters_bytes(int T, int H, int I, int E, int k) {
+  if (decode_scratch_bytes(T, H, I, E, k) == 0) return 0;
+  return dec::dec_scratch(T, H, I, E, k, dec::hbuf_per_tile(T)).p1;
+}
+
 // Batches of up to four tokens run on the CUDA-core kernel, larger ones on the tensor-core one.
 int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
