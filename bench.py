@@ -51,6 +51,29 @@ def expert_bytes(H: int, I: int) -> int:
     return codes + scales
 
 
+PROFILE = os.path.join(ROOT, "profiles", "moe_decode_gemv_kernel_olmoe_decode.md")
+PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_gemv.cu",
+                   "quantized_mixture_experts_grouped_b200/csrc/decode_common.cuh"]
+
+
+def profiled_traffic():
+    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu summary,
+    or None when the summary is missing or the kernel's sources changed since the capture."""
+    import hashlib
+    import re
+    try:
+        text = open(PROFILE).read()
+        digest = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read()
+                                         for f in PROFILE_SOURCES)).hexdigest()[:16]
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel source hash \([^)]*\): ([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch: ([0-9]+)", text)
+    if not m_hash or not m_tr or m_hash.group(1) != digest:
+        return None
+    return int(m_tr.group(1))
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -418,8 +441,9 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(config_of(wl, args, args.path), us_per_layer=ms_total / args.steps / wl.layers * 1e3),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": achieved / hbm_peak, "traffic": None,
-                     "kernel": "one moe_w4a16_layer launch sequence per layer (event pair per layer)",
+                     "frac": achieved / hbm_peak,
+                     "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
+                     "kernel": "moe_decode_gemv_kernel (the one launch per layer; event pair per layer)",
                      "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,
                      "peak_kind": f"{peaks_kind} HBM copy"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d_bytes(),
@@ -442,9 +466,14 @@ def main():
     ap.add_argument("--workload", default="olmoe_decode", choices=["olmoe_decode"])
     ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="fewer layers than the workload's (profiling runs only; the metric uses 16)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = mi.WORKLOADS[args.workload]
+    if args.layers is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, layers=max(1, args.layers))
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
