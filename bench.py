@@ -457,13 +457,244 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- one-layer workloads
+
+def cpu_baseline_tokens(wl: mi.Workload, budget_s: float = 12.0):
+    """Oracle tokens/s for a one-layer workload over a bounded sample of its tokens (the layer's
+    experts packed by the oracle; tokens taken in order until about budget_s of work)."""
+    import oracle
+    logits = mi.router_logits(wl, 0, 0)
+    idx, wts = oracle.route(logits, wl.k)
+    layer = OracleLayer(wl, 0, sorted(set(idx.ravel().tolist())))
+    x = mi.activations(wl, 0, 0)
+    threads = max(1, os.cpu_count() or 1)
+    done, t_used, n = 0, 0.0, 1
+    while t_used < budget_s and done < wl.T:
+        toks = np.arange(done, min(wl.T, done + n), dtype=np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_ffn(x, idx, wts, layer.w13, layer.s13, layer.w2, layer.s2, wl.H, wl.I, tokens=toks,
+                       n_threads=threads)
+        t_used += time.perf_counter() - t0
+        done += len(toks)
+        n = min(2 * n, 64)
+    return {"value": done / t_used, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"the first {done} of the {wl.T} tokens of one {wl.name} layer ({t_used:.1f} s of oracle "
+                      f"work, experts packed by the oracle)"}
+
+
+def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
+    """Large-batch workloads (prefill, large expert): one layer of T tokens per step through
+    moe_w4a16_layer (route, permute, gather, two grouped GEMMs, combine)."""
+    import quantized_mixture_experts_grouped_b200 as q
+    device = torch.device("cuda", local)
+    H, I, E, k, T = wl.H, wl.I, wl.E, wl.k, wl.T
+    w13b, w2b = mi.device_bank_weights(wl, 0, device)
+    w13, s13 = q.alloc_bank(E, 2 * I, H, device)
+    w2, s2 = q.alloc_bank(E, H, I, device)
+    q.moe_quantize_pack(w13b, w13, s13)
+    q.moe_quantize_pack(w2b, w2, s2)
+    del w13b, w2b
+    x_host = torch.from_numpy(mi.activations(wl, 0, 0).view(np.int16)).view(torch.bfloat16).pin_memory()
+    lg_host = torch.from_numpy(mi.router_logits(wl, 0, 0).view(np.int16)).view(torch.bfloat16).pin_memory()
+    x, lg = x_host.to(device), lg_host.to(device)
+    idx = torch.empty((T, k), dtype=torch.int32, device=device)
+    wts = torch.empty((T, k), dtype=torch.float32, device=device)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
+    out_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    ws = q.alloc_workspace(T, H, I, E, k, device)
+    flags = q.PATHS[args.path]
+    s = torch.cuda.Stream(device)
+    peaks, peaks_kind = load_peaks()
+    sampler = ClockSampler(local)
+
+    def call(xx, ll):
+        q.moe_w4a16_layer(xx, ll, k, w13, s13, w2, s2, H, I, idx, wts, ws, out, flags=flags, stream=s)
+
+    with torch.cuda.stream(s):
+        n0 = q.moe_launch_count()
+        call(x, lg)
+        launches = q.moe_launch_count() - n0
+        for _ in range(args.warmup):
+            call(x, lg)
+        s.synchronize()
+        sampler.start()
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 1.0:
+            call(x, lg)
+            s.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(args.steps):
+            call(x, lg)
+        e1.record(s)
+        e1.synchronize()
+        barrier(world)
+        clocks = sampler.stop()
+        ms = all_max(e0.elapsed_time(e1), world) / args.steps
+        # end to end: inputs from pinned host memory, output back to the host, every step
+        for _ in range(args.warmup):
+            x.copy_(x_host, non_blocking=True); lg.copy_(lg_host, non_blocking=True)
+            call(x, lg)
+            out_host.copy_(out, non_blocking=True)
+        s.synchronize()
+        barrier(world)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s)
+        for _ in range(args.steps):
+            x.copy_(x_host, non_blocking=True); lg.copy_(lg_host, non_blocking=True)
+            call(x, lg)
+            out_host.copy_(out, non_blocking=True)
+            s.synchronize()
+        f1.record(s)
+        f1.synchronize()
+        e2e_ms = all_max(f0.elapsed_time(f1), world) / args.steps
+    status = q.moe_workspace_status(ws, s)
+    if rank != 0:
+        return
+    flops = 6.0 * H * I * T * k
+    achieved = flops / (ms / 1e3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = {
+        "metric": METRIC, "value": T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(wl, args, args.path), us_per_layer=ms * 1e3,
+                       l2="inputs larger than L2 (packed bank of the layer)"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "whole layer (route, permute, gather, gate/up and down grouped GEMMs, combine): "
+                               "6*H*I*T*k flop over the layer's event-timed duration",
+                     "peak_kind": f"{peaks_kind} bf16 dense (burst)"},
+        "e2e": {"value": T * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": (x.numel() + lg.numel()) * 2, "d2h_bytes_per_step": out.numel() * 2},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_tokens(wl)
+    print(json.dumps(line), flush=True)
+
+
+def run_slots(args, wl: mi.Workload, rank: int, world: int, local: int):
+    """Batched decode through the GPU slot cache: every layer keeps S of its E experts on the
+    device, the rest in a pinned host bank; each layer call routes, reads the routed set back to
+    the host, refills misses by cudaMemcpyAsync on a copy stream and runs the FFN in waves."""
+    import quantized_mixture_experts_grouped_b200 as q
+    device = torch.device("cuda", local)
+    H, I, E, k, T, S, Ls = wl.H, wl.I, wl.E, wl.k, wl.T, wl.slots, wl.layers
+    caches = []
+    for l in range(Ls):
+        w13b, w2b = mi.device_bank_weights(wl, l, device)
+        d13, ds13 = q.alloc_bank(E, 2 * I, H, device)
+        d2, ds2 = q.alloc_bank(E, H, I, device)
+        q.moe_quantize_pack(w13b, d13, ds13)
+        q.moe_quantize_pack(w2b, d2, ds2)
+        del w13b, w2b
+        bank = q.alloc_bank(E, 2 * I, H, pinned=True) + q.alloc_bank(E, H, I, pinned=True)
+        for hst, dev in zip(bank, (d13, ds13, d2, ds2)):
+            hst.copy_(dev)
+        del d13, ds13, d2, ds2
+        pool = q.alloc_bank(S, 2 * I, H, device) + q.alloc_bank(S, H, I, device)
+        caches.append(q.SlotCache(E, S, H, I, bank, pool))
+    torch.cuda.synchronize()
+    R = 8    # distinct step inputs, replayed cyclically
+    xs = torch.stack([torch.stack([torch.from_numpy(mi.activations(wl, l, r).view(np.int16)) for l in range(Ls)])
+                      for r in range(R)]).view(torch.bfloat16).to(device)
+    lgs = torch.stack([torch.stack([torch.from_numpy(mi.router_logits(wl, l, r).view(np.int16)) for l in range(Ls)])
+                       for r in range(R)]).view(torch.bfloat16).to(device)
+    steps_total = args.warmup + args.steps
+    idx_all = torch.empty((steps_total, Ls, T, k), dtype=torch.int32, device=device)
+    wts = torch.empty((T, k), dtype=torch.float32, device=device)
+    out = torch.empty((Ls, T, H), dtype=torch.bfloat16, device=device)
+    wave_tables = torch.empty(E * ((E + S - 1) // S + 1), dtype=torch.int32, device=device)
+    ws = q.alloc_workspace(T, H, I, E, k, device)
+    s, cs = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    flags = q.PATHS[args.path]
+    loads = [0]
+    waves = [0]
+
+    def step(i):
+        r = i % R
+        for l in range(Ls):
+            nw, nl = caches[l].layer(xs[r, l], lgs[r, l], k, idx_all[i, l], wts, wave_tables, ws, out[l], flags,
+                                     stream=s, copy_stream=cs)
+            loads[0] += nl
+            waves[0] += nw
+
+    # pinned host -> device copy bandwidth of this box (the bound of the refills)
+    big_h = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    big_d = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(cs):
+        for _ in range(2):
+            big_d.copy_(big_h, non_blocking=True)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        c0.record(cs)
+        for _ in range(4):
+            big_d.copy_(big_h, non_blocking=True)
+        c1.record(cs)
+        c1.synchronize()
+    h2d_peak = 4 * big_h.numel() / (c0.elapsed_time(c1) / 1e3) / 1e9
+    del big_h, big_d
+    sampler = ClockSampler(local)
+    with torch.cuda.stream(s):
+        for i in range(args.warmup):
+            step(i)
+        s.synchronize()
+        loads[0] = waves[0] = 0
+        n0 = q.moe_launch_count()
+        sampler.start()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for i in range(args.warmup, steps_total):
+            step(i)
+        e1.record(s)
+        e1.synchronize()
+        clocks = sampler.stop()
+        ms = all_max(e0.elapsed_time(e1), world) / args.steps
+        launches = (q.moe_launch_count() - n0) // args.steps
+    status = q.moe_workspace_status(ws, s)
+    if rank != 0:
+        return
+    idx_h = idx_all[args.warmup:].cpu().numpy()
+    needed = sum(len(np.unique(idx_h[i, l])) for i in range(args.steps) for l in range(Ls))
+    h2d_bytes = loads[0] * expert_bytes(H, I)
+    h2d_gbs = h2d_bytes / (args.steps * ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(wl, args, args.path), us_per_layer=ms / Ls * 1e3,
+                       l2="pinned host bank of all layers, 16 device slots per layer"),
+        "slot_cache": {"hit_rate": 1.0 - loads[0] / max(1, needed), "misses_per_layer_step": loads[0] / (args.steps * Ls),
+                       "distinct_per_layer_step": needed / (args.steps * Ls), "waves_per_layer_step": waves[0] / (args.steps * Ls),
+                       "h2d_gbs": h2d_gbs, "h2d_peak_gbs": h2d_peak},
+        "roofline": {"bound": "h2d", "achieved": h2d_gbs, "peak": h2d_peak, "unit": "GB/s",
+                     "frac": h2d_gbs / h2d_peak, "traffic": None,
+                     "kernel": "refill copies (cudaMemcpyAsync, pinned host -> slot pool) over the step time",
+                     "peak_kind": "pinned host-to-device copy measured in this run"},
+        "e2e": {"value": T * world / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes // args.steps,
+                "d2h_bytes_per_step": Ls * 8 * ((E + 63) // 64)},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="olmoe_decode", choices=["olmoe_decode"])
+    ap.add_argument("--workload", default="olmoe_decode",
+                    choices=["olmoe_decode", "olmoe_slots", "olmoe_prefill", "large_expert"])
     ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
@@ -478,6 +709,10 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, wl, rank, world)
+        elif wl.T > 16:
+            run_single_layer(args, wl, rank, world, local)
+        elif wl.slots:
+            run_slots(args, wl, rank, world, local)
         else:
             run_ours(args, wl, rank, world, local)
     finally:

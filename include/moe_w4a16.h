@@ -126,8 +126,9 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  * configurable GPU-resident slot cache and fused grouped MoE kernels"):
  *   y_e(x) = W2_e . ( silu(W_gate_e . x) * (W_up_e . x) ),  silu(z) = z / (1 + exp(-z))
  *   out[t] = sum_{j<k} wts[t][j] * y_{idx[t][j]}(x_t)
- * with W = q * s dequantised from the packed banks. Products run on bf16 operands with fp32
- * accumulation; the intermediate h is rounded to bf16; out is bf16.
+ * with W = q * s dequantised from the packed banks. The tensor-core paths multiply bf16
+ * operands (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the CUDA-core decode
+ * kernel (fused path, T <= 4) keeps the products and h in fp32. out is bf16.
  *   x: bf16 [T][H]; idx, wts: the router's outputs [T][k].
  *   w13/s13: packed W13 ([2I][H]) per slot, w2/s2: packed W2 ([H][I]) per slot;
  *     slot stride = moe_packed_bytes / moe_scales_count of the matrix.
