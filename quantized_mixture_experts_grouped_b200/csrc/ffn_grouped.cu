@@ -28,7 +28,8 @@ namespace moe {
 namespace {
 
 constexpr int kGStages = 4;
-constexpr int kGThreads = 448;
+constexpr int kGThreads = 480;      // 15 warps
+constexpr int kGIssuer1 = 14;       // second MMA-issuing warp (block 1 of the pair)
 constexpr int kGEpi0 = 2;           // warps 2..5
 constexpr int kGDq0 = 6;            // warps 6..13
 constexpr int kTokTile = 128;
@@ -52,7 +53,7 @@ struct GSmem {
   uint64_t afull[2], aempty[2];
   uint64_t dfull, dempty;
   uint64_t tq_full[4], tq_empty[4];
-  uint64_t drain;
+  uint64_t drain[2];
   int tq[4];
   uint32_t tmem_base;
   int abort;
@@ -141,13 +142,14 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
   if (tid == 0) {
     for (int i = 0; i < kGStages; ++i) {
       tc::mbar_init(&s.full[i], 1);
-      tc::mbar_init(&s.empty[i], 8 + 1);       // 8 dequant warps + the MMA commit
+      tc::mbar_init(&s.empty[i], 8 + 2);       // 8 dequant warps + the two issuers' commits
     }
-    for (int i = 0; i < 2; ++i) { tc::mbar_init(&s.afull[i], 8); tc::mbar_init(&s.aempty[i], 1); }
-    tc::mbar_init(&s.dfull, 1);
+    for (int i = 0; i < 2; ++i) { tc::mbar_init(&s.afull[i], 8); tc::mbar_init(&s.aempty[i], 2); }
+    tc::mbar_init(&s.dfull, 2);
     tc::mbar_init(&s.dempty, 4);
-    for (int i = 0; i < 4; ++i) { tc::mbar_init(&s.tq_full[i], 1); tc::mbar_init(&s.tq_empty[i], 1 + 4 + 8); }
-    tc::mbar_init(&s.drain, 1);
+    for (int i = 0; i < 4; ++i) { tc::mbar_init(&s.tq_full[i], 1); tc::mbar_init(&s.tq_empty[i], 2 + 4 + 8); }
+    tc::mbar_init(&s.drain[0], 1);
+    tc::mbar_init(&s.drain[1], 1);
     s.abort = 0;
     tc::fence_barrier_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(&xmap) : "memory");
@@ -214,8 +216,12 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
         tc::mbar_wait(&s.full[j % kGStages], (j / kGStages) & 1, &never);
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == kGIssuer1) {
+    // ---------------------------------------------------------------- MMA issuers
+    // issuer `me` runs the MMAs of block `me` of the pair into accumulator D_me: one MMA
+    // costs its issuing thread about as much as its tensor-pipe time at these N, so two
+    // issuers keep the pipe fed
+    const int me = warp == 1 ? 0 : 1;
     if (lane == 0) {
       int it = 0, a_it = 0;
       for (int n = 0;; ++n) {
@@ -239,14 +245,12 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
           }
           tc::tc_fence_after();
           const uint32_t bbase = tc::smem_u32(s.st[st].b[0]);
-          const uint32_t a0 = tmem + kGA + ab * 128, a1 = a0 + 64;
+          const uint32_t a = tmem + kGA + ab * 128 + me * 64, dacc = tmem + (me ? kGD1 : kGD0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t baddr = bbase + (kk >> 2) * kBBoxBytes + (kk & 3) * 32;
             const uint64_t bdesc = tc::smem_desc(baddr, 16, 1024, 2);
-            const uint32_t acc = (g > 0 || kk > 0) ? 1u : 0u;
-            tc::mma_ts(tmem + kGD0, a0 + kk * 8, bdesc, idesc, acc);
-            tc::mma_ts(tmem + kGD1, a1 + kk * 8, bdesc, idesc, acc);
+            tc::mma_ts(dacc, a + kk * 8, bdesc, idesc, (g > 0 || kk > 0) ? 1u : 0u);
           }
           tc::mma_commit(&s.aempty[ab]);
           tc::mma_commit(&s.empty[st]);
@@ -258,12 +262,12 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
         }
         tc::mma_commit(&s.dfull);
       }
-      tc::mma_commit(&s.drain);
+      tc::mma_commit(&s.drain[me]);
       volatile int never = 0;
-      tc::mbar_wait(&s.drain, 0, &never);
+      tc::mbar_wait(&s.drain[me], 0, &never);
     }
     __syncwarp();
-  } else if (warp >= kGDq0) {
+  } else if (warp >= kGDq0 && warp < kGDq0 + 8) {
     // ---------------------------------------------------------------- dequantisers -> TMEM
     const int quarter = warp & 3, blk = (warp - kGDq0) >> 2;     // block 0 or 1 of the pair
     const int r = quarter * 32 + lane;
@@ -351,11 +355,9 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             if (j < cn) {
-              const int pos = d.p0 + c0 + j;
-              const float w = P.wts[P.perm[pos]];
-              uint16_t* o = P.out + (size_t)pos * P.out_ld;
-              o[col0] = __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(v0[j])));
-              o[col1] = __bfloat16_as_ushort(__float2bfloat16_rn(w * __uint_as_float(v1[j])));
+              uint16_t* o = P.out + (size_t)(d.p0 + c0 + j) * P.out_ld;
+              o[col0] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v0[j])));
+              o[col1] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v1[j])));
             }
           }
         }
@@ -408,8 +410,10 @@ __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t* __restric
   }
 }
 
-// out[t] = bf16( acc + sum_j yw[inv[t][j]] ) with yw already weighted (bf16), fixed j order.
+// out[t] = bf16( acc + sum_j wts[t][j] * y[inv[t][j]] ) over the bf16 down-projection rows y,
+// in fixed j order.
 __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __restrict__ yw,
+                                                           const float* __restrict__ wts,
                                                            const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ inv,
                                                            const int32_t* __restrict__ table, int H, int k,
@@ -424,12 +428,13 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __res
   for (int i = 0; i < 8; ++i) v[i] = accumulate ? accp[i] : 0.f;
   for (int j = 0; j < k; ++j) {
     if (slot_of(table, idx[(size_t)t * k + j]) < 0) continue;
+    const float w = wts[(size_t)t * k + j];
     const uint4 y = *reinterpret_cast<const uint4*>(yw + (size_t)inv[(size_t)t * k + j] * H + n0);
     const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] += bf16_bits_to_float(yy[i] & 0xffffu);
-      v[2 * i + 1] += bf16_bits_to_float(yy[i] >> 16);
+      v[2 * i] = fmaf(w, bf16_bits_to_float(yy[i] & 0xffffu), v[2 * i]);
+      v[2 * i + 1] = fmaf(w, bf16_bits_to_float(yy[i] >> 16), v[2 * i + 1]);
     }
   }
   if (out) {
@@ -531,7 +536,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   int32_t* list_dn = list_gu + L.tile_list_len;
   uint16_t* xp = reinterpret_cast<uint16_t*>(a.ws + L.xp);
   uint16_t* hp = reinterpret_cast<uint16_t*>(a.ws + L.hp);
-  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // weighted y, bf16
+  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // y per pair, bf16
   int* ctl = reinterpret_cast<int*>(a.ws + L.status);
 
   if (int rc = launch_permute(a.idx, a.T, a.k, a.E, counts, offsets, perm, inv,
@@ -564,7 +569,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   if (int rc = launch_gemm(P, hmap, max_chunks * HP, s)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
-  combine_bf16_kernel<<<grid, 256, 0, s>>>(yw, a.idx, inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
+  combine_bf16_kernel<<<grid, 256, 0, s>>>(yw, a.wts, a.idx, inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
                                            a.accumulate, a.out);
   return check_launch("combine_bf16_kernel");
 }
