@@ -25,9 +25,12 @@
 #include "tc.cuh"
 
 namespace moe {
+namespace dec {
+extern unsigned long long* g_trace;   // diagnostics buffer (moe_debug_set_decode_trace)
+}
 namespace {
 
-constexpr int kGStages = 4;
+constexpr int kGStages = 3;
 constexpr int kGThreads = 480;      // 15 warps
 constexpr int kGIssuer1 = 14;       // second MMA-issuing warp (block 1 of the pair)
 constexpr int kGEpi0 = 2;           // warps 2..5
@@ -49,6 +52,7 @@ struct __align__(1024) GStage {
 
 struct GSmem {
   GStage st[kGStages];
+  uint16_t ostage[128][256];    // epilogue: the tile's outputs, token-major (bf16, 64 KB)
   uint64_t full[kGStages], empty[kGStages];
   uint64_t afull[2], aempty[2];
   uint64_t dfull, dempty;
@@ -70,6 +74,7 @@ struct GParams {
   const int32_t* ntiles;                    // total tile count (device)
   const int32_t* offsets;                   // grouped pair offsets [E+1]
   const int32_t* table;                     // expert -> slot (nullable)
+  unsigned long long* trace;                // optional per-CTA clock stamps (diagnostics)
   const int32_t* perm;                      // pair id of grouped position
   const float* wts;                         // router weights [T*k]
   uint16_t* out;                            // gate/up: Hp [Tk][I]; down: Yp [Tk][H] (weighted)
@@ -102,6 +107,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
       : "r"(taddr)
       : "memory");
+}
+
+// diagnostics: 7 reference (after set-up); first tile of the CTA, K group g < 16:
+// 48+g stage issued, 16+g dequantised A ready (warp 6), 32+g issuer 0 done issuing;
+// 1 epilogue saw D of tile 0, 2 epilogue released D of tile 0, 3 issuer 0 starts tile 1
+__device__ __forceinline__ void gtrace(const GParams& P, int slot) {
+  if (P.trace) P.trace[blockIdx.x * 64 + slot] = (unsigned long long)clock64();
+}
+
+// Named barrier over `n` threads that also ANDs a flag over them (uniform decisions).
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\t"
+               "selp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(n) : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -163,6 +184,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
   const uint32_t tmem = s.tmem_base;
   volatile int* abort = &s.abort;
   const int total = *P.ntiles;
+  if (tid == 0) gtrace(P, 7);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
@@ -200,6 +222,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
           tc::bulk_g2s(S.w[1], wb + t1 * kTileBytes, 8192, &s.full[st], pol_w);
           tc::bulk_g2s(S.sc[0], sb + t0 * kRowBlock, 256, &s.full[st], pol_w);
           tc::bulk_g2s(S.sc[1], sb + t1 * kRowBlock, 256, &s.full[st], pol_w);
+          if (it < 16) gtrace(P, 48 + it);
         }
       }
       if (!ok) {
@@ -235,6 +258,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
         const uint32_t idesc = tc::idesc_bf16_f32(128, nmma);
         if (!tc::mbar_wait(&s.dempty, (n & 1) ^ 1, abort)) { report_status(P.ctl, MOE_ERR_TIMEOUT, 24); break; }
         tc::tc_fence_after();
+        if (me == 0 && n == 1) gtrace(P, 3);
         bool ok = true;
         for (int g = 0; g < P.G; ++g, ++it, ++a_it) {
           const int st = it % kGStages, ab = a_it & 1;
@@ -254,6 +278,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
           }
           tc::mma_commit(&s.aempty[ab]);
           tc::mma_commit(&s.empty[st]);
+          if (me == 0 && a_it < 16) gtrace(P, 32 + a_it);
         }
         if (!ok) {
           report_status(P.ctl, MOE_ERR_TIMEOUT, 25);
@@ -316,6 +341,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&s.afull[ab]);
+        if (warp == kGDq0 && lane == 0 && a_it < 16) gtrace(P, 16 + a_it);
       }
       if (!ok) break;
     }
@@ -326,45 +352,73 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int n = 0;; ++n) {
       const int q = n & 3;
-      if (!gwait(&s.tq_full[q], (n >> 2) & 1, abort)) break;
+      // every exit is decided by all four epilogue warps together (they meet at named barriers)
+      if (!bar_and(1, 128, gwait(&s.tq_full[q], (n >> 2) & 1, abort))) break;
       const int packed = s.tq[q];
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.tq_empty[q]);
       if (packed < 0) break;
       const TileDesc d = describe(P, packed);
-      if (!gwait(&s.dfull, n & 1, abort)) break;
+      if (!bar_and(1, 128, gwait(&s.dfull, n & 1, abort))) break;
       tc::tc_fence_after();
+      if (warp == kGEpi0 && lane == 0 && n == 0) gtrace(P, 1);
+      // the whole tile: tensor memory -> registers -> shared memory (token-major, bf16); the
+      // accumulators are released as soon as they are read, so the next tile's MMAs overlap the
+      // 16-byte coalesced stores of whole output rows below
+      const int etid = tid - kGEpi0 * 32;
       for (int c0 = 0; c0 < d.ntok; c0 += 32) {
         uint32_t v0[32], v1[32];
         tmem_ld32(trow + kGD0 + c0, v0);
         tmem_ld32(trow + kGD1 + c0, v1);
         tc::tmem_wait_ld();
-        const int cn = min(32, d.ntok - c0);
         if (P.mode == kModeGateUp) {
-          const size_t col = d.bp * kRowBlock + r;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            if (j < cn) {
-              const float g = __uint_as_float(v0[j]), u = __uint_as_float(v1[j]);
-              const float h = g / (1.f + expf(-g)) * u;
-              P.out[(size_t)(d.p0 + c0 + j) * P.out_ld + col] = __bfloat16_as_ushort(__float2bfloat16_rn(h));
-            }
+            // silu(g) * u with the hardware exp and reciprocal: h is rounded to bf16 (8 bits)
+            // right after, far coarser than their few-ulp fp32 error
+            const float g = __uint_as_float(v0[j]), u = __uint_as_float(v1[j]);
+            s.ostage[c0 + j][r] = __bfloat16_as_ushort(__float2bfloat16_rn(__fdividef(g * u, 1.f + __expf(-g))));
           }
         } else {
-          const size_t col0 = d.rb0 * kRowBlock + r, col1 = d.rb1 * kRowBlock + r;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            if (j < cn) {
-              uint16_t* o = P.out + (size_t)(d.p0 + c0 + j) * P.out_ld;
-              o[col0] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v0[j])));
-              o[col1] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v1[j])));
-            }
+            s.ostage[c0 + j][r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v0[j])));
+            s.ostage[c0 + j][kRowBlock + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v1[j])));
           }
         }
       }
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.dempty);
+      if (warp == kGEpi0 && lane == 0 && n == 0) gtrace(P, 2);
+      tc::named_bar_sync(1, 128);               // the staged tile is complete
+      if (P.mode == kModeGateUp) {
+        // 128 columns = 16 pieces of 16 bytes per token row; a warp stores two rows per step
+        const size_t col = (size_t)d.bp * kRowBlock + (etid & 15) * 8;
+        for (int t0 = 0; t0 < d.ntok; t0 += 32) {
+          uint4 v[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) v[m] = *reinterpret_cast<const uint4*>(&s.ostage[t0 + (etid >> 4) + 8 * m][(etid & 15) * 8]);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int t = t0 + (etid >> 4) + 8 * m;
+            if (t < d.ntok) *reinterpret_cast<uint4*>(P.out + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
+          }
+        }
+      } else {
+        // 256 columns = 32 pieces per token row; a warp stores one whole row per step
+        const size_t col = d.rb0 * kRowBlock + (etid & 31) * 8;
+        for (int t0 = 0; t0 < d.ntok; t0 += 16) {
+          uint4 v[4];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) v[m] = *reinterpret_cast<const uint4*>(&s.ostage[t0 + (etid >> 5) + 4 * m][(etid & 31) * 8]);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int t = t0 + (etid >> 5) + 4 * m;
+            if (t < d.ntok) *reinterpret_cast<uint4*>(P.out + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
+          }
+        }
+      }
     }
   }
 
@@ -560,12 +614,14 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   P.K = a.H; P.G = a.H / kGroup; P.rows_half = a.I; P.mode = kModeGateUp;
   P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
   P.perm = perm; P.wts = a.wts; P.out = hp; P.out_ld = a.I; P.Tk = Tk; P.ctl = ctl;
+  P.trace = nullptr;
   if (int rc = launch_gemm(P, xmap, max_chunks * IB, s)) return rc;
 
   P.w = a.w2; P.s = a.s2;
   P.w_stride = (size_t)a.H * a.I / 2; P.s_stride = (size_t)a.H * (a.I / kGroup);
   P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
   P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;
+  P.trace = dec::g_trace;
   if (int rc = launch_gemm(P, hmap, max_chunks * HP, s)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
