@@ -361,6 +361,17 @@ class DecodeBench:
         self.out_host.copy_(self.out_e2e, non_blocking=True)
         self.stream.synchronize()           # the host reads the step's result
 
+    def distinct_experts_mean(self) -> float:
+        """Mean number of distinct experts the ring's logits select per layer (top-k by bf16 logit
+        descending, id ascending): the experts whose packed bytes one layer launch must read."""
+        wl, tot = self.wl, 0
+        for r in range(self.RING):
+            for l in range(wl.layers):
+                lg = mi.bf16_bits_to_f32(mi.router_logits(wl, l, r))
+                order = np.lexsort((np.broadcast_to(np.arange(wl.E), lg.shape), -lg), axis=-1)[:, :wl.k]
+                tot += len(np.unique(order))
+        return tot / (self.RING * wl.layers)
+
     def run(self, graphs, n, start=0):
         for i in range(n):
             graphs[(start + i) % self.RING].replay()
@@ -432,7 +443,7 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         return
     tokens = wl.T * args.steps * world
     value = tokens / (ms_total / 1e3)
-    bytes_per_layer = 8 * expert_bytes(wl.H, wl.I) if wl.T == 1 else None
+    bytes_per_layer = bench.distinct_experts_mean() * expert_bytes(wl.H, wl.I)
     achieved = bytes_per_layer / (layer_ms / 1e3) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     line = {
@@ -443,7 +454,9 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
                      "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
-                     "kernel": "moe_decode_gemv_kernel (the one launch per layer; event pair per layer)",
+                     "kernel": ("moe_decode_gemv_kernel" if wl.T <= 4 else "moe_decode_kernel")
+                               + " (the one launch per layer; event pair per layer)"
+                               if args.path in ("auto", "decode") else "all launches of the layer (event pair per layer)",
                      "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,
                      "peak_kind": f"{peaks_kind} HBM copy"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d_bytes(),
@@ -695,16 +708,21 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="olmoe_decode",
                     choices=["olmoe_decode", "olmoe_slots", "olmoe_prefill", "large_expert"])
-    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped", "sequential"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers than the workload's (profiling runs only; the metric uses 16)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per step other than the workload's (ablations; the metric uses the default)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     wl = mi.WORKLOADS[args.workload]
     if args.layers is not None:
         import dataclasses
         wl = dataclasses.replace(wl, layers=max(1, args.layers))
+    if args.tokens is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, T=max(1, args.tokens))
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":

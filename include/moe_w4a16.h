@@ -54,7 +54,7 @@ enum {
   MOE_PATH_SIMPLE = 1,     /* CUDA-core grouped kernels (reference path, any size)            */
   MOE_PATH_DECODE = 2,     /* one fused launch: dequant on the fly, tcgen05, in-kernel combine */
   MOE_PATH_GROUPED = 3,    /* permute + tcgen05 grouped GEMMs (gate/up, down) + combine       */
-  MOE_PATH_SEQUENTIAL = 4, /* one expert at a time through the grouped kernels (ablation)     */
+  MOE_PATH_SEQUENTIAL = 4, /* one expert at a time through the same kernels (ablation)        */
   MOE_PATH_MASK = 0xff,
   MOE_FLAG_ACCUMULATE = 0x100 /* add this call's contribution into the workspace fp32
                                  accumulator instead of starting from zero (slot-cache waves) */

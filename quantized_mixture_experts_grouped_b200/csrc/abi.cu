@@ -58,6 +58,7 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
   L.hp = take(sizeof(uint16_t) * Tk * I);
   L.yp = take(sizeof(float) * Tk * H);
   L.acc = take(sizeof(float) * (size_t)T * H);
+  L.seq = take(sizeof(int32_t) * (size_t)E * E);
   L.dec = take(decode_scratch_bytes(T, H, I, E, k));
   L.total = off;
   return L;

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
 
-FFN_PATHS = ["simple", "decode", "grouped"]
+FFN_PATHS = ["simple", "decode", "grouped", "sequential"]
 
 
 def _supported(path, T, k):
@@ -219,7 +219,7 @@ def test_ffn_edge_cases_small_batch(path):
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
 
 
-@pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped"])
+@pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped", "sequential"])
 @pytest.mark.parametrize("T", [1, 5, 16, 300])
 def test_layer_call_routes_and_runs(path, T):
     """moe_w4a16_layer: routing (in-kernel on the fused path) + FFN in one call."""
