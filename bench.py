@@ -682,6 +682,8 @@ def run_slots(args, wl: mi.Workload, rank: int, world: int, local: int):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(config_of(wl, args, args.path), us_per_layer=ms / Ls * 1e3,
                        l2="pinned host bank of all layers, 16 device slots per layer"),
+        "memory": {"slot_pool_bytes": Ls * S * expert_bytes(H, I), "pinned_bank_bytes": Ls * E * expert_bytes(H, I),
+                   "resident_fraction": S / E, "device_peak_reserved_bytes": torch.cuda.max_memory_reserved(device)},
         "slot_cache": {"hit_rate": 1.0 - loads[0] / max(1, needed), "misses_per_layer_step": loads[0] / (args.steps * Ls),
                        "distinct_per_layer_step": needed / (args.steps * Ls), "waves_per_layer_step": waves[0] / (args.steps * Ls),
                        "h2d_gbs": h2d_gbs, "h2d_peak_gbs": h2d_peak},
