@@ -94,7 +94,31 @@ int launch_gather_rows(const uint16_t* x, const int32_t* perm, int Tk, int k, in
                        cudaStream_t s);
 int launch_combine(const FfnArgs& a, const WsLayout& L, cudaStream_t s);
 
+// Launch with programmatic stream serialisation (PDL): the kernel may start while the previous
+// one on the stream finishes; every kernel launched this way calls pdl_begin() first.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- device helpers ----
+// Start of a PDL-launched kernel: wait until the previous kernel's results are visible, then let
+// the next kernel start launching (it waits for this one the same way).
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
 __device__ __forceinline__ int slot_of(const int32_t* table, int e) { return table ? table[e] : e; }

@@ -160,6 +160,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (tid == 0) {
     for (int i = 0; i < kGStages; ++i) {
       tc::mbar_init(&s.full[i], 1);
@@ -444,6 +445,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
 __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t* __restrict__ counts, int E,
                                                         const int32_t* __restrict__ table, int pairs,
                                                         int32_t* __restrict__ list, int32_t* __restrict__ total) {
+  pdl_begin();
   const int e = blockIdx.x;
   __shared__ int base, mine;
   if (threadIdx.x == 0) {
@@ -473,6 +475,7 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __res
                                                            const int32_t* __restrict__ table, int H, int k,
                                                            float* __restrict__ acc, bool accumulate,
                                                            uint16_t* __restrict__ out) {
+  pdl_begin();
   const int t = blockIdx.x;
   const int n0 = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
   if (n0 >= H) return;
@@ -598,10 +601,14 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
     return rc;
   if (int rc = launch_gather_rows(a.x, perm, Tk, a.k, a.H, xp, s)) return rc;
   const int IB = a.I / kRowBlock, HP = a.H / 256;
-  tile_list_kernel<<<a.E, 256, 0, s>>>(counts, a.E, a.slot, IB, list_gu, tiles + 0);
-  if (int rc = check_launch("tile_list_kernel")) return rc;
-  tile_list_kernel<<<a.E, 256, 0, s>>>(counts, a.E, a.slot, HP, list_dn, tiles + 1);
-  if (int rc = check_launch("tile_list_kernel")) return rc;
+  note_launch();
+  if (int rc = check_cuda(launch_pdl(tile_list_kernel, dim3(a.E), dim3(256), 0, s, (const int32_t*)counts, a.E, a.slot,
+                                     IB, list_gu, tiles + 0), "tile_list_kernel"))
+    return rc;
+  note_launch();
+  if (int rc = check_cuda(launch_pdl(tile_list_kernel, dim3(a.E), dim3(256), 0, s, (const int32_t*)counts, a.E, a.slot,
+                                     HP, list_dn, tiles + 1), "tile_list_kernel"))
+    return rc;
   const int max_chunks = (Tk + kTokTile - 1) / kTokTile + a.E;
 
   CUtensorMap xmap, hmap;
@@ -625,9 +632,11 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   if (int rc = launch_gemm(P, hmap, max_chunks * HP, s)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
-  combine_bf16_kernel<<<grid, 256, 0, s>>>(yw, a.wts, a.idx, inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
-                                           a.accumulate, a.out);
-  return check_launch("combine_bf16_kernel");
+  note_launch();
+  return check_cuda(launch_pdl(combine_bf16_kernel, grid, dim3(256), 0, s, (const uint16_t*)yw, a.wts, a.idx,
+                               (const int32_t*)inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
+                               a.accumulate, a.out),
+                    "combine_bf16_kernel");
 }
 
 }  // namespace moe

@@ -26,6 +26,7 @@ constexpr int kMaxPerLane = kMaxExperts / 32;
 
 __global__ void __launch_bounds__(128) route_kernel(const uint16_t* __restrict__ logits, int T, int E, int k,
                                                     int32_t* __restrict__ idx, float* __restrict__ wts) {
+  pdl_begin();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -94,6 +95,7 @@ constexpr int kChunk = 1024;   // pairs per permute block
 // scratch: chunk_counts [nb][E] then chunk_base [nb][E]
 __global__ void __launch_bounds__(kChunk) perm_count_kernel(const int32_t* __restrict__ idx, int Tk, int E,
                                                             int32_t* __restrict__ chunk_counts) {
+  pdl_begin();
   __shared__ int cnt[kMaxExperts];
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
@@ -110,6 +112,7 @@ __global__ void __launch_bounds__(kMaxExperts) perm_scan_kernel(int nb, int E, c
                                                                 int32_t* __restrict__ chunk_base,
                                                                 int32_t* __restrict__ counts,
                                                                 int32_t* __restrict__ offsets) {
+  pdl_begin();
   __shared__ int tot[kMaxExperts];
   const int e = threadIdx.x;
   int run = 0;
@@ -140,6 +143,7 @@ __global__ void __launch_bounds__(kMaxExperts) perm_scan_kernel(int nb, int E, c
 __global__ void __launch_bounds__(kChunk) perm_place_kernel(const int32_t* __restrict__ idx, int Tk, int E,
                                                             const int32_t* __restrict__ chunk_base,
                                                             int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  pdl_begin();
   __shared__ int wcount[kChunk / 32][kMaxExperts];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < (kChunk / 32) * E; i += blockDim.x) wcount[i / E][i % E] = 0;
@@ -162,6 +166,7 @@ __global__ void __launch_bounds__(kChunk) perm_place_kernel(const int32_t* __res
 
 __global__ void gather_rows_kernel(const uint16_t* __restrict__ x, const int32_t* __restrict__ perm, int k, int H,
                                    uint16_t* __restrict__ xp) {
+  pdl_begin();
   const int pos = blockIdx.x;
   const int t = perm[pos] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
@@ -178,8 +183,9 @@ size_t permute_scratch_count(int T, int k, int E) {
 
 int launch_route(const uint16_t* logits, int T, int E, int k, int32_t* idx, float* wts, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  route_kernel<<<ceil_div(T, 4), 128, 0, s>>>(logits, T, E, k, idx, wts);
-  return check_launch("route_kernel");
+  note_launch();
+  return check_cuda(launch_pdl(route_kernel, dim3(ceil_div(T, 4)), dim3(128), 0, s, logits, T, E, k, idx, wts),
+                    "route_kernel");
 }
 
 int launch_permute(const int32_t* idx, int T, int k, int E, int32_t* counts, int32_t* offsets, int32_t* perm,
@@ -189,22 +195,30 @@ int launch_permute(const int32_t* idx, int T, int k, int E, int32_t* counts, int
   int32_t* chunk_counts = scratch;
   int32_t* chunk_base = scratch + (size_t)nb * E;
   if (nb > 0) {
-    perm_count_kernel<<<nb, kChunk, 0, s>>>(idx, Tk, E, chunk_counts);
-    if (int rc = check_launch("perm_count_kernel")) return rc;
+    note_launch();
+    if (int rc = check_cuda(launch_pdl(perm_count_kernel, dim3(nb), dim3(kChunk), 0, s, idx, Tk, E, chunk_counts),
+                            "perm_count_kernel"))
+      return rc;
   }
-  perm_scan_kernel<<<1, kMaxExperts, 0, s>>>(nb, E, chunk_counts, chunk_base, counts, offsets);
-  if (int rc = check_launch("perm_scan_kernel")) return rc;
+  note_launch();
+  if (int rc = check_cuda(launch_pdl(perm_scan_kernel, dim3(1), dim3(kMaxExperts), 0, s, nb, E,
+                                     (const int32_t*)chunk_counts, chunk_base, counts, offsets),
+                          "perm_scan_kernel"))
+    return rc;
   if (nb > 0) {
-    perm_place_kernel<<<nb, kChunk, 0, s>>>(idx, Tk, E, chunk_base, perm, inv);
-    if (int rc = check_launch("perm_place_kernel")) return rc;
+    note_launch();
+    if (int rc = check_cuda(launch_pdl(perm_place_kernel, dim3(nb), dim3(kChunk), 0, s, idx, Tk, E,
+                                       (const int32_t*)chunk_base, perm, inv),
+                            "perm_place_kernel"))
+      return rc;
   }
   return MOE_OK;
 }
 
 int launch_gather_rows(const uint16_t* x, const int32_t* perm, int Tk, int k, int H, uint16_t* xp, cudaStream_t s) {
   if (Tk == 0) return MOE_OK;
-  gather_rows_kernel<<<Tk, 128, 0, s>>>(x, perm, k, H, xp);
-  return check_launch("gather_rows_kernel");
+  note_launch();
+  return check_cuda(launch_pdl(gather_rows_kernel, dim3(Tk), dim3(128), 0, s, x, perm, k, H, xp), "gather_rows_kernel");
 }
 
 }  // namespace moe
