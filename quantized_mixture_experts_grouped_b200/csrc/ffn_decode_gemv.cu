@@ -98,15 +98,14 @@ __device__ __forceinline__ void tile_dot(uint4 wv, float s, const float* xb, uin
 }
 
 // sum over c = c0..c1 (in that order) of partial entry (base + c), rows q*32 + lane of each
-// quarter q, tokens t < T: the loads of up to kBatch entries are issued before any is summed.
-template <int TT>
+// quarter q, tokens t < T: the loads of up to KB entries are issued before any is summed.
+template <int TT, int KB>
 __device__ __forceinline__ void sum_partials(const float* P0, int base, int c0, int c1, int T, int lane,
                                              float (&acc)[4][TT]) {
-  constexpr int kBatch = 8 / TT;
-  for (int cb = c0; cb <= c1; cb += kBatch) {
-    float v[kBatch][4][TT];
+  for (int cb = c0; cb <= c1; cb += KB) {
+    float v[KB][4][TT];
 #pragma unroll
-    for (int e = 0; e < kBatch; ++e) {
+    for (int e = 0; e < KB; ++e) {
       const float* pp = P0 + (size_t)(base + cb + e) * T * kRowBlock + lane;
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -115,11 +114,43 @@ __device__ __forceinline__ void sum_partials(const float* P0, int base, int c0, 
           v[e][q][t] = (cb + e <= c1 && t < T) ? __ldcg(pp + t * kRowBlock + q * 32) : 0.f;
     }
 #pragma unroll
-    for (int e = 0; e < kBatch; ++e)
+    for (int e = 0; e < KB; ++e)
 #pragma unroll
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int t = 0; t < TT; ++t) acc[q][t] += v[e][q][t];
+  }
+}
+
+// The same for two ranges at once (gate and up partials of a feature block): each round issues
+// the loads of up to KB entries of both before summing, each range in its own order.
+template <int TT, int KB>
+__device__ __forceinline__ void sum_partials2(const float* P0, int ba, int a0, int a1, float (&acc_a)[4][TT], int bb,
+                                              int b0, int b1, float (&acc_b)[4][TT], int T, int lane) {
+  for (int r = 0; a0 + r * KB <= a1 || b0 + r * KB <= b1; ++r) {
+    float va[KB][4][TT], vb[KB][4][TT];
+#pragma unroll
+    for (int e = 0; e < KB; ++e) {
+      const int ca = a0 + r * KB + e, cb = b0 + r * KB + e;
+      const float* pa = P0 + (size_t)(ba + ca) * T * kRowBlock + lane;
+      const float* pb = P0 + (size_t)(bb + cb) * T * kRowBlock + lane;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          va[e][q][t] = (ca <= a1 && t < T) ? __ldcg(pa + t * kRowBlock + q * 32) : 0.f;
+          vb[e][q][t] = (cb <= b1 && t < T) ? __ldcg(pb + t * kRowBlock + q * 32) : 0.f;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < KB; ++e)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          acc_a[q][t] += va[e][q][t];
+          acc_b[q][t] += vb[e][q][t];
+        }
   }
 }
 
@@ -404,8 +435,8 @@ __global__ void __launch_bounds__(kGThreads, 1) moe_decode_gemv_kernel(const __g
           for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int t = 0; t < TT; ++t) { g[q][t] = 0.f; up[q][t] = 0.f; }
-          sum_partials<TT>(P.p1, Rg, pl.first1(Rg), pl.last1(Rg), T, lane, g);
-          sum_partials<TT>(P.p1, Ru, pl.first1(Ru), pl.last1(Ru), T, lane, up);
+          sum_partials2<TT, (TT == 1 ? 4 : 1)>(P.p1, Rg, pl.first1(Rg), pl.last1(Rg), g, Ru, pl.first1(Ru),
+                                                pl.last1(Ru), up, T, lane);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -425,7 +456,7 @@ __global__ void __launch_bounds__(kGThreads, 1) moe_decode_gemv_kernel(const __g
           for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int t = 0; t < TT; ++t) yo[q][t] = 0.f;
-          sum_partials<TT>(P.p2, key, pl.first2(key), pl.last2(key), T, lane, yo);
+          sum_partials<TT, 16 / TT>(P.p2, key, pl.first2(key), pl.last2(key), T, lane, yo);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
 #pragma unroll
