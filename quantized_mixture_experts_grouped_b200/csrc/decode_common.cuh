@@ -100,51 +100,67 @@ __device__ __forceinline__ uint32_t route_key(uint32_t bits, int e) {
 }
 
 // Routes token t with one warp (same selection rule as the stand-alone router: bf16 logit
-// descending, expert id ascending). The chosen logits are decoded back from the winning keys;
-// the renormalised weight of choice j is exp(l_j - l_max) / sum over the k chosen, which equals
-// the full softmax renormalised over the chosen experts.
-__device__ inline void route_token(RouteSmem& rs, const DecParams& P, int t, int lane) {
+// descending, expert id ascending). Lane l holds the keys of experts l, l+32, ...; each of the
+// k rounds takes the warp maximum of the keys (unique: the id is in them) and retires it. The
+// chosen logits are decoded back from the winning keys; the renormalised weight of choice j is
+// exp(l_j - l_max) / sum over the k chosen (= the full softmax renormalised over the chosen),
+// with the exponentials taken after the selection, one per lane.
+template <int kPer>
+__device__ inline void route_token_n(RouteSmem& rs, const DecParams& P, int t, int lane) {
   const int E = P.E, k = P.k;
   const uint16_t* lt = P.logits + (size_t)t * E;
-  constexpr int kPer = kMaxExperts / 32;
   uint32_t key[kPer];
+  if (lane == 0 && t == 0) trace_clk(P, 13);
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
     key[i] = (e < E) ? route_key(lt[e], e) : 0u;
   }
-  float mx = 0.f, el[kPer];    // lane (j % 32) keeps exp(l_j - l_max) of choice j in el[j / 32]
+  if (t == 0 && __shfl_sync(kFull, key[0], 0) != 1u && lane == 0) trace_clk(P, 14);
+  uint32_t mine[8];    // lane (j % 32) keeps the winning key of choice j in mine[j / 32]
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) el[i] = 0.f;
+  for (int i = 0; i < 8; ++i) mine[i] = 0;
+  uint32_t first = 0;
   for (int j = 0; j < k; ++j) {
-    uint32_t best = 0;
+    uint32_t best = key[0];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) best = max(best, key[i]);
+    for (int i = 1; i < kPer; ++i) best = max(best, key[i]);
     const uint32_t win = __reduce_max_sync(kFull, best);
 #pragma unroll
     for (int i = 0; i < kPer; ++i)
-      if (key[i] == win) key[i] = 0;                  // keys are unique (the id is in them)
-    const int e = 0xffff - (int)(win & 0xffffu);
-    const uint32_t ord = win >> 16;
-    const float lw = bf16_bits_to_float((ord & 0x8000u) ? (ord & 0x7fffu) : (~ord & 0xffffu));
-    if (j == 0) mx = lw;
-    if ((j & 31) == lane) {
-      rs.idx[t * k + j] = e;
+      if (key[i] == win) key[i] = 0;
+    if (j == 0) first = win;
 #pragma unroll
-      for (int i = 0; i < kPer; ++i)
-        if ((j >> 5) == i) el[i] = expf(lw - mx);
-    }
+    for (int i = 0; i < 8; ++i)
+      if ((j & 31) == lane && (j >> 5) == i) mine[i] = win;
   }
-  float sum = 0.f;
+  if (lane == 0 && t == 0) trace_clk(P, 15);
+  auto logit_of = [](uint32_t w) {
+    const uint32_t ord = w >> 16;
+    return bf16_bits_to_float((ord & 0x8000u) ? (ord & 0x7fffu) : (~ord & 0xffffu));
+  };
+  const float mx = logit_of(first);
+  float el[8], sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) sum += el[i];
+  for (int i = 0; i < 8; ++i) {
+    const int j = 32 * i + lane;
+    el[i] = j < k ? expf(logit_of(mine[i]) - mx) : 0.f;
+    sum += el[i];
+    if (j < k) rs.idx[t * k + j] = 0xffff - (int)(mine[i] & 0xffffu);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const int j = 32 * i + lane;
     if (j < k) rs.wts[t * k + j] = el[i] / sum;
   }
+}
+
+__device__ inline void route_token(RouteSmem& rs, const DecParams& P, int t, int lane) {
+  if (P.E <= 64) route_token_n<2>(rs, P, t, lane);
+  else if (P.E <= 128) route_token_n<4>(rs, P, t, lane);
+  else route_token_n<8>(rs, P, t, lane);
 }
 
 // Clears the routing state (before the dependency wait; no global reads).

@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kGThreads, 1) moe_decode_gemv_kernel(const __g
           for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int t = 0; t < TT; ++t) yo[q][t] = 0.f;
-          sum_partials<TT, 16 / TT>(P.p2, key, pl.first2(key), pl.last2(key), T, lane, yo);
+          sum_partials<TT, (TT == 1 ? 12 : 8 / TT)>(P.p2, key, pl.first2(key), pl.last2(key), T, lane, yo);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
 #pragma unroll
