@@ -29,7 +29,7 @@ namespace moe {
 namespace dec {
 namespace {
 
-constexpr int kGWarps = 18;                // warp 0 producer, warps 1..16 compute, 17 epilogue
+constexpr int kGWarps = 19;                // warp 0 producer, warps 1..16 compute, 17..18 epilogue
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kGComputeWarps = 16;
 constexpr int kGEpiWarp = 17;
@@ -385,9 +385,12 @@ __global__ void __launch_bounds__(kGThreads, 1) moe_decode_gemv_kernel(const __g
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue warp
-    // per block, in the compute warps' order: quarter sums -> this CTA's partial; the arrival
-    // that completes a block does its reduction (h of a feature block, or an output row block).
+    // ------------------------------------------------------------ epilogue warps
+    // epilogue warp ew takes the blocks written to quarter-sum buffer ew (every other block), so
+    // the reductions of consecutive blocks run side by side: quarter sums -> this CTA's partial;
+    // the arrival that completes a block does its reduction (h of a feature block, or an output
+    // row block).
+    const int ew = warp - kGEpiWarp;
     int nblk = 0, nh = 0;
     for (int phase = 1; phase <= 2; ++phase) {
       const int ub = phase == 1 ? pl.b1 : pl.b2, ue = phase == 1 ? pl.e1 : pl.e2;
@@ -396,6 +399,7 @@ __global__ void __launch_bounds__(kGThreads, 1) moe_decode_gemv_kernel(const __g
       bool stop = false;
       for (int key = ub / per; key <= (ue - 1) / per; ++key, ++nblk) {
         const int b = nblk & 1;
+        if (b != ew) continue;
         if (!warp_wait(&s.redfull[b], (nblk >> 1) & 1, abort)) { stop = true; break; }
         float y[4][TT];
 #pragma unroll
