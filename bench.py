@@ -51,8 +51,8 @@ def expert_bytes(H: int, I: int) -> int:
     return codes + scales
 
 
-PROFILE = os.path.join(ROOT, "profiles", "moe_decode_gemv_kernel_olmoe_decode.md")
-PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_gemv.cu",
+PROFILE = os.path.join(ROOT, "profiles", "moe_decode_mma_kernel_olmoe_decode.md")
+PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_mma.cu",
                    "quantized_mixture_experts_grouped_b200/csrc/decode_common.cuh"]
 
 
@@ -454,9 +454,9 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
                      "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
-                     "kernel": ("moe_decode_gemv_kernel" if wl.T <= 4 else "moe_decode_kernel")
+                     "kernel": ("moe_decode_kernel" if args.path == "decode_tc" else "moe_decode_mma_kernel")
                                + " (the one launch per layer; event pair per layer)"
-                               if args.path in ("auto", "decode") else "all launches of the layer (event pair per layer)",
+                               if args.path in ("auto", "decode", "decode_tc") else "all launches of the layer (event pair per layer)",
                      "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,
                      "peak_kind": f"{peaks_kind} HBM copy"},
         "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d_bytes(),
@@ -710,7 +710,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="olmoe_decode",
                     choices=["olmoe_decode", "olmoe_slots", "olmoe_prefill", "large_expert"])
-    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped", "sequential"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "decode_tc", "grouped", "sequential"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers than the workload's (profiling runs only; the metric uses 16)")

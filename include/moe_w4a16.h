@@ -52,9 +52,11 @@ enum {
 enum {
   MOE_PATH_AUTO = 0,       /* fused decode kernel for small batches, grouped GEMM otherwise   */
   MOE_PATH_SIMPLE = 1,     /* CUDA-core grouped kernels (reference path, any size)            */
-  MOE_PATH_DECODE = 2,     /* one fused launch: dequant on the fly, tcgen05, in-kernel combine */
+  MOE_PATH_DECODE = 2,     /* one fused launch (T <= 16): routing, both projections on the
+                              int8 warp-MMA path, in-kernel combine                          */
   MOE_PATH_GROUPED = 3,    /* permute + tcgen05 grouped GEMMs (gate/up, down) + combine       */
   MOE_PATH_SEQUENTIAL = 4, /* one expert at a time through the same kernels (ablation)        */
+  MOE_PATH_DECODE_TC = 5,  /* the fused launch with bf16 tcgen05 MMAs (T <= 16; comparison)   */
   MOE_PATH_MASK = 0xff,
   MOE_FLAG_ACCUMULATE = 0x100 /* add this call's contribution into the workspace fp32
                                  accumulator instead of starting from zero (slot-cache waves) */
@@ -126,9 +128,10 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  * configurable GPU-resident slot cache and fused grouped MoE kernels"):
  *   y_e(x) = W2_e . ( silu(W_gate_e . x) * (W_up_e . x) ),  silu(z) = z / (1 + exp(-z))
  *   out[t] = sum_{j<k} wts[t][j] * y_{idx[t][j]}(x_t)
- * with W = q * s dequantised from the packed banks. The tensor-core paths multiply bf16
- * operands (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the CUDA-core decode
- * kernel (fused path, T <= 4) keeps the products and h in fp32. out is bf16.
+ * with W = q * s dequantised from the packed banks. The tcgen05 paths multiply bf16 operands
+ * (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the default fused decode kernel
+ * (T <= 16) multiplies the codes exactly with x and h held as 16-bit fixed point per
+ * 128-element group (error <= max|group| / 65278), scales applied in fp32. out is bf16.
  *   x: bf16 [T][H]; idx, wts: the router's outputs [T][k].
  *   w13/s13: packed W13 ([2I][H]) per slot, w2/s2: packed W2 ([H][I]) per slot;
  *     slot stride = moe_packed_bytes / moe_scales_count of the matrix.

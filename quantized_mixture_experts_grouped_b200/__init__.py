@@ -19,9 +19,10 @@ LIB_PATH = os.path.join(_HERE, "libmoe_w4a16.so")
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 0, 1, 2, 3, 4
 MOE_PATH_AUTO, MOE_PATH_SIMPLE, MOE_PATH_DECODE, MOE_PATH_GROUPED, MOE_PATH_SEQUENTIAL = 0, 1, 2, 3, 4
+MOE_PATH_DECODE_TC = 5
 MOE_FLAG_ACCUMULATE = 0x100
 PATHS = {"auto": MOE_PATH_AUTO, "simple": MOE_PATH_SIMPLE, "decode": MOE_PATH_DECODE,
-         "grouped": MOE_PATH_GROUPED, "sequential": MOE_PATH_SEQUENTIAL}
+         "grouped": MOE_PATH_GROUPED, "sequential": MOE_PATH_SEQUENTIAL, "decode_tc": MOE_PATH_DECODE_TC}
 
 
 class MoeError(RuntimeError):

@@ -81,6 +81,7 @@ struct FfnArgs {
   bool accumulate;
   const uint16_t* logits; // fused decode: route in-kernel when non-null
   int32_t* idx_out; float* wts_out;
+  bool tc_decode;         // fused decode on the tcgen05 kernel instead of the warp-MMA one
 };
 int ffn_simple(const FfnArgs& a, cudaStream_t s);
 int ffn_sequential(const FfnArgs& a, cudaStream_t s);

@@ -88,6 +88,7 @@ struct RouteSmem {
   uint32_t present[kMaxExperts / 32];
   uint32_t tokbits[kMaxT][kMaxExperts / 32];
   int act[kMaxExperts];
+  int sl[kMaxExperts];      // slot of act[j]
   int nact;
   int over;
 };
@@ -206,6 +207,7 @@ __device__ inline void route_finish(RouteSmem& rs, const DecParams& P, int tid, 
       int a = __popc(rs.present[w] & ((1u << (tid & 31)) - 1u));
       for (int i = 0; i < w; ++i) a += __popc(rs.present[i]);
       rs.act[a] = tid;
+      rs.sl[a] = slot_of(P.slot, tid);
     }
   }
   if (tid == 0) {
@@ -403,12 +405,11 @@ inline bool split_fits(int T, int H, int I, int E, int k, int grid) {
 int num_sms();
 extern unsigned long long* g_trace;
 
-// CUDA-core decode kernel for T <= kGemvMaxT (defined in ffn_decode_gemv.cu)
-constexpr int kGemvMaxT = 4;
-size_t gemv_hbuf_per_tile(int T);
-size_t gemv_smem_bytes(int T, int H);
-int gemv_stages(int T, int H);
-int launch_decode_gemv(const DecParams& P, int grid, cudaStream_t s);
+// Warp-MMA decode kernel for T <= kMmaMaxT (defined in ffn_decode_mma.cu)
+constexpr int kMmaMaxT = 16;
+size_t mma_hbuf_per_tile(int T);
+int mma_stages(int T, int H);
+int launch_decode_mma(const DecParams& P, int grid, cudaStream_t s);
 
 }  // namespace dec
 }  // namespace moe

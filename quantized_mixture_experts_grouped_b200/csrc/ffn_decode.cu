@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         if (!warp_wait(&s.empty[st], ((it / NS) & 1) ^ 1, abort)) { ok = false; break; }
         int j, lt;
         pl.locate(phase, u, j, lt);
-        const int sl = slot_of(P.slot, s.rs.act[j]);
+        const int sl = s.rs.sl[j];
         const uint8_t* wsrc = phase == 1 ? P.w13 + (size_t)sl * w13_bytes : P.w2 + (size_t)sl * w2_bytes;
         const uint16_t* ssrc = phase == 1 ? P.s13 + (size_t)sl * s13_count : P.s2 + (size_t)sl * s2_count;
         if (lane == 0) tc::mbar_arrive_expect_tx(&s.full[st], (uint32_t)(n * (kTileBytes + kRowBlock * 2)));
@@ -518,7 +518,7 @@ int decode_stages(int H) {
 size_t decode_smem_bytes(int H) { return fixed_smem_bytes(H) + (size_t)decode_stages(H) * kStageBytes; }
 
 // h bytes per (selected expert, K group of I): the larger of the two kernels' layouts
-size_t hbuf_per_tile(int T) { return std::max<size_t>(2 * kHTile, gemv_hbuf_per_tile(std::min(T, kGemvMaxT))); }
+size_t hbuf_per_tile(int T) { return std::max<size_t>(2 * kHTile, mma_hbuf_per_tile(std::min(T, kMmaMaxT))); }
 
 int launch_tensor(const DecParams& P0, int grid, cudaStream_t s) {
   DecParams P = P0;
@@ -560,7 +560,7 @@ bool ffn_decode_supported(const FfnArgs& a) {
         a.I % kRowBlock == 0 && a.H > 0 && a.I > 0))
     return false;
   if (!dec::split_fits(a.T, a.H, a.I, a.E, a.k, dec::kMaxGrid)) return false;
-  return a.T <= dec::kGemvMaxT ? dec::gemv_stages(a.T, a.H) >= 2 : dec::decode_stages(a.H) >= 2;
+  return (a.T <= dec::kMmaMaxT && !a.tc_decode) ? dec::mma_stages(a.T, a.H) >= 2 : dec::decode_stages(a.H) >= 2;
 }
 
 size_t decode_scratch_bytes(int T, int H, int I, int E, int k) {
@@ -574,7 +574,7 @@ size_t decode_counters_bytes(int T, int H, int I, int E, int k) {
   return dec::dec_scratch(T, H, I, E, k, dec::hbuf_per_tile(T)).p1;
 }
 
-// Batches of up to four tokens run on the CUDA-core kernel, larger ones on the tensor-core one.
+// Batches of up to sixteen tokens run on the warp-MMA kernel unless the tcgen05 one is asked for.
 int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
   const dec::DecScratch D = dec::dec_scratch(a.T, a.H, a.I, a.E, a.k, dec::hbuf_per_tile(a.T));
@@ -599,7 +599,7 @@ int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   const int m_max = std::min(a.E, a.T * a.k);
   const long tiles1 = (long)m_max * 2 * (a.I / kRowBlock) * (a.H / kGroup);
   const int grid = (int)std::max<long>(1, std::min<long>(std::min(dec::num_sms(), dec::kMaxGrid), tiles1));
-  return a.T <= dec::kGemvMaxT ? dec::launch_decode_gemv(P, grid, s) : dec::launch_tensor(P, grid, s);
+  return (a.T <= dec::kMmaMaxT && !a.tc_decode) ? dec::launch_decode_mma(P, grid, s) : dec::launch_tensor(P, grid, s);
 }
 
 }  // namespace moe

@@ -18,17 +18,17 @@ pytestmark = pytest.mark.gpu
 
 q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
 
-FFN_PATHS = ["simple", "decode", "grouped", "sequential"]
+FFN_PATHS = ["simple", "decode", "decode_tc", "grouped", "sequential"]
 
 
 def _supported(path, T, k):
     """The fused decode path takes small batches only (T <= 16 and T*k <= 256)."""
-    if path == "decode" and not (1 <= T <= 16 and T * k <= 256):
+    if path in ("decode", "decode_tc") and not (1 <= T <= 16 and T * k <= 256):
         pytest.skip("fused decode path is for small batches")
 
 
 def _supported_h(path, H):
-    if path == "decode" and H > 3072:
+    if path in ("decode", "decode_tc") and H > 3072:
         pytest.skip("fused decode path stages the activations in shared memory: H <= 3072")
     if path == "grouped" and H % 256:
         pytest.skip("grouped GEMM pairs 128-row blocks of W2: H must be a multiple of 256")
@@ -219,7 +219,7 @@ def test_ffn_edge_cases_small_batch(path):
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
 
 
-@pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped", "sequential"])
+@pytest.mark.parametrize("path", ["auto", "decode", "decode_tc", "simple", "grouped", "sequential"])
 @pytest.mark.parametrize("T", [1, 5, 16, 300])
 def test_layer_call_routes_and_runs(path, T):
     """moe_w4a16_layer: routing (in-kernel on the fused path) + FFN in one call."""
