@@ -51,8 +51,8 @@ def expert_bytes(H: int, I: int) -> int:
     return codes + scales
 
 
-PROFILE = os.path.join(ROOT, "profiles", "moe_decode_mma_kernel_olmoe_decode.md")
-PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_mma.cu",
+PROFILE = os.path.join(ROOT, "profiles", "moe_decode_rows_kernel_olmoe_decode.md")
+PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_rows.cu",
                    "quantized_mixture_experts_grouped_b200/csrc/decode_common.cuh"]
 
 
@@ -454,7 +454,8 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
                      "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
-                     "kernel": ("moe_decode_kernel" if args.path == "decode_tc" else "moe_decode_mma_kernel")
+                     "kernel": ("moe_decode_kernel" if args.path == "decode_tc" else
+                                ("moe_decode_rows_kernel" if wl.T == 1 else "moe_decode_mma_kernel"))
                                + " (the one launch per layer; event pair per layer)"
                                if args.path in ("auto", "decode", "decode_tc") else "all launches of the layer (event pair per layer)",
                      "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,

@@ -42,7 +42,8 @@ struct DecParams {
   int* ctl;
   int* hcnt;                    // [selected expert][I/128] phase-1 arrivals per feature block
   int* fcnt;                    // [H/128] phase-2 arrivals per output row block
-  int* hdone;                   // [0] feature blocks finished, [1] CTAs finished
+  int* hdone;                   // [0] feature blocks finished, [1] CTAs finished, [2..3] as u64:
+                                // running count of CTAs past phase 1 (single-token kernel)
   float* p1;                    // phase-1 partials: [row block + CTA][T][128]
   float* p2;                    // phase-2 partials: [output block + CTA][T][128]
   uint8_t* hbuf;                // h operand tiles (layout depends on the kernel)
@@ -377,6 +378,49 @@ __device__ inline void finish_launch(const Plan& pl, const DecParams& P, volatil
   }
 }
 
+// ---- warp-level int8 MMA pieces (decode kernels on the mma.sync path)
+// D (16 x 8, s32) += A (16 x 32, u8) * B (32 x 8, s8).
+__device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                     uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte position of element e (0..7) of a word in the permuted order (0, 4, 1, 5, 2, 6, 3, 7).
+__device__ __forceinline__ int perm_pos(int e) { return ((e & 3) << 1) | (e >> 2); }
+
+// Encodes one 128-element group of one token as two B-operand columns. Lane l holds elements
+// q * 32 + l (q = 0..3) in v[q]. hi / lo: the columns (bytes), starting at the group's first
+// word; rec: the group's record {8 * sum(v) over elements 0..63, a, 8 * sum(v) over 64..127, a}.
+// Called by a whole warp; generic pointers (shared or global memory).
+__device__ __forceinline__ void encode_group(const float (&v)[4], uint8_t* hi, uint8_t* lo, int4* rec, int lane) {
+  float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+  const float inv = mx > 0.f ? 32639.f / mx : 0.f;
+  int sum0 = 0, sum1 = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int iv = max(-32639, min(32639, __float2int_rn(v[q] * inv)));
+    const int h8 = (iv + 128) >> 8, l8 = iv - 256 * h8;
+    const int k = q * 32 + lane, at = (k >> 3) * 8 + perm_pos(k & 7);
+    hi[at] = (uint8_t)h8;
+    lo[at] = (uint8_t)l8;
+    if (q < 2) sum0 += iv; else sum1 += iv;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sum0 += __shfl_xor_sync(kFull, sum0, o);
+    sum1 += __shfl_xor_sync(kFull, sum1, o);
+  }
+  if (lane == 0) {
+    const int a = __float_as_int(mx * (1.f / 32639.f));
+    *rec = make_int4(8 * sum0, a, 8 * sum1, a);
+  }
+}
+
 // ---- host side
 struct DecScratch { size_t hcnt, fcnt, hdone, p1, p2, hbuf, total; };
 // hbuf_per_tile: bytes of h operand per (selected expert, K group of I)
@@ -387,7 +431,7 @@ inline DecScratch dec_scratch(int T, int H, int I, int E, int k, size_t hbuf_per
   auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 256); return at; };
   D.hcnt = take(sizeof(int) * m * nI);
   D.fcnt = take(sizeof(int) * nH);
-  D.hdone = take(sizeof(int) * 2);
+  D.hdone = take(sizeof(int) * 4);
   D.p1 = take(sizeof(float) * (m * 2 * nI + kMaxGrid) * T * kRowBlock);
   D.p2 = take(sizeof(float) * (nH + kMaxGrid) * T * kRowBlock);
   D.hbuf = take(m * nI * hbuf_per_tile);
@@ -404,6 +448,11 @@ inline bool split_fits(int T, int H, int I, int E, int k, int grid) {
 
 int num_sms();
 extern unsigned long long* g_trace;
+
+// Single-token decode kernel (defined in ffn_decode_rows.cu)
+bool rows_supported(int T, int H, int I, int E, int k);
+size_t rows_hbuf_bytes(int H, int I, int E, int k);
+int launch_decode_rows(const DecParams& P, int grid, cudaStream_t s);
 
 // Warp-MMA decode kernel for T <= kMmaMaxT (defined in ffn_decode_mma.cu)
 constexpr int kMmaMaxT = 16;

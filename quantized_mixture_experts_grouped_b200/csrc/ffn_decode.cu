@@ -574,7 +574,8 @@ size_t decode_counters_bytes(int T, int H, int I, int E, int k) {
   return dec::dec_scratch(T, H, I, E, k, dec::hbuf_per_tile(T)).p1;
 }
 
-// Batches of up to sixteen tokens run on the warp-MMA kernel unless the tcgen05 one is asked for.
+// One token runs on the single-token kernel, up to sixteen on the warp-MMA kernel, unless the
+// tcgen05 one is asked for.
 int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   const WsLayout L = ws_layout(a.T, a.H, a.I, a.E, a.k);
   const dec::DecScratch D = dec::dec_scratch(a.T, a.H, a.I, a.E, a.k, dec::hbuf_per_tile(a.T));
@@ -599,7 +600,9 @@ int ffn_decode(const FfnArgs& a, cudaStream_t s) {
   const int m_max = std::min(a.E, a.T * a.k);
   const long tiles1 = (long)m_max * 2 * (a.I / kRowBlock) * (a.H / kGroup);
   const int grid = (int)std::max<long>(1, std::min<long>(std::min(dec::num_sms(), dec::kMaxGrid), tiles1));
-  return (a.T <= dec::kMmaMaxT && !a.tc_decode) ? dec::launch_decode_mma(P, grid, s) : dec::launch_tensor(P, grid, s);
+  if (a.tc_decode || a.T > dec::kMmaMaxT) return dec::launch_tensor(P, grid, s);
+  if (dec::rows_supported(a.T, a.H, a.I, a.E, a.k)) return dec::launch_decode_rows(P, dec::num_sms(), s);
+  return dec::launch_decode_mma(P, grid, s);
 }
 
 }  // namespace moe

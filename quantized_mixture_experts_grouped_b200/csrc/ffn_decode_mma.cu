@@ -58,47 +58,6 @@ struct __align__(128) MSmem {
   // their group records [H/128][4 NB] x 16 B and the stage ring
 };
 
-__device__ __forceinline__ void imma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                     uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Byte position of element e (0..7) of a word in the permuted order (0, 4, 1, 5, 2, 6, 3, 7).
-__device__ __forceinline__ int perm_pos(int e) { return ((e & 3) << 1) | (e >> 2); }
-
-// Encodes one 128-element group of one token as two B-operand columns. Lane l holds elements
-// q * 32 + l (q = 0..3) in v[q]. hi / lo: the columns (bytes), starting at the group's first
-// word; rec: the group's record {8 * sum(v) over elements 0..63, a, 8 * sum(v) over 64..127, a}.
-// Called by a whole warp; generic pointers (shared or global memory).
-__device__ __forceinline__ void encode_group(const float (&v)[4], uint8_t* hi, uint8_t* lo, int4* rec, int lane) {
-  float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
-  const float inv = mx > 0.f ? 32639.f / mx : 0.f;
-  int sum0 = 0, sum1 = 0;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int iv = max(-32639, min(32639, __float2int_rn(v[q] * inv)));
-    const int h8 = (iv + 128) >> 8, l8 = iv - 256 * h8;
-    const int k = q * 32 + lane, at = (k >> 3) * 8 + perm_pos(k & 7);
-    hi[at] = (uint8_t)h8;
-    lo[at] = (uint8_t)l8;
-    if (q < 2) sum0 += iv; else sum1 += iv;
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    sum0 += __shfl_xor_sync(kFull, sum0, o);
-    sum1 += __shfl_xor_sync(kFull, sum1, o);
-  }
-  if (lane == 0) {
-    const int a = __float_as_int(mx * (1.f / 32639.f));
-    *rec = make_int4(8 * sum0, a, 8 * sum1, a);
-  }
-}
-
 // One 128 x 128 tile for compute warp (mt, kh): rows mt*16 + g and + 8, K half kh, lane (g, c).
 // tile_issue loads the operands and issues the MMAs; tile_finish adds the tile's contribution,
 // so that the next tile's MMAs can be issued before this one's results are needed.
