@@ -131,7 +131,8 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  * with W = q * s dequantised from the packed banks. The tcgen05 paths multiply bf16 operands
  * (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the default fused decode kernel
  * (T <= 16) multiplies the codes exactly with x and h held as 16-bit fixed point per
- * 128-element group (error <= max|group| / 65278), scales applied in fp32. out is bf16.
+ * 128-element group (32 for h at T = 1; error <= max|group| / 65278), scales applied in fp32.
+ * out is bf16.
  *   x: bf16 [T][H]; idx, wts: the router's outputs [T][k].
  *   w13/s13: packed W13 ([2I][H]) per slot, w2/s2: packed W2 ([H][I]) per slot;
  *     slot stride = moe_packed_bytes / moe_scales_count of the matrix.

@@ -11,7 +11,10 @@
 //    slices, computes the complete gate and up sums, and writes h = w * silu(gate) * up of its
 //    features, already encoded as the down projection's B operand (16-bit fixed point per
 //    32-feature slice, two s8 columns: the MMA k-step of phase 2 is exactly one slice);
-//  * one counter: every CTA adds 1 after its slices are written; phase 2 waits for all;
+//  * one counter: every CTA adds 1 after its slices are written and phase 2 waits until the
+//    launch's G arrivals are in. The counter only grows (64-bit): a launch's base is its value
+//    at the start rounded down to a multiple of G (arrivals of the same launch are < G), so no
+//    CTA resets it and no exit atomic is needed;
 //  * phase 2 (down): a CTA takes 16 output rows over every selected expert and all of I, so the
 //    router-weighted sum over experts and K ends in its own registers and shared memory, and the
 //    bf16 output is written directly. Its W2 rows are in shared memory before h is ready.
@@ -38,7 +41,7 @@ constexpr int kRData = 32768;             // weight bytes per stage
 constexpr int kRScales = 1024;            // scale bytes per stage
 constexpr int kRStage = kRData + kRScales;
 constexpr int kSliceF = 32;               // features per phase-1 slice (= one phase-2 k-step)
-constexpr int kSliceB = 72;               // encoded h slice: hi and lo columns (32 B each), {a, 8 sum v}
+constexpr int kSliceB = 72;               // encoded h slice: hi and lo columns (32 B each), {a, a * 8 sum v}
 constexpr int kORows = 16;                // output rows per phase-2 block
 constexpr int kXPad = 32;                 // bytes after each activation column
 
@@ -49,11 +52,21 @@ struct __align__(128) RSmem {
   RouteSmem rs;
   float red1[2][8][2 * kSliceF];          // [buffer][K part][gate rows, up rows]
   float red2[kRCompute][kORows];          // [warp][row] phase-2 sums
+  float wsel[kMaxExperts];                // router weight of selected expert j
   int abort;
   // followed in dynamic shared memory by the activation columns [2][H + kXPad] (bytes) and their
   // group records [H/128] x 16 B, the encoded h [m][I/32] x kSliceB, and the stage ring (on a
   // 1024-byte boundary)
 };
+
+// D = A * B (zero accumulator), the m16n8k32 u8 x s8 -> s32 warp MMA.
+__device__ __forceinline__ void imma0(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                      uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
 
 // 4-D tensor load: box at coordinates (x, 0, block, slot) of `map` into shared memory.
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int block, int slot,
@@ -64,6 +77,15 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, i
       ::"r"(tc::smem_u32(dst)), "l"(map), "r"(x), "r"(0), "r"(block), "r"(slot), "r"(tc::smem_u32(bar)),
         "l"(policy)
       : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // The split of both phases, identical in every CTA.
@@ -120,25 +142,31 @@ __global__ void __launch_bounds__(kRThreads, 1)
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) trace_at(P, 0);
-  // activations as B-operand columns (one token): warp w encodes K groups w, w + 18, ...; the
-  // loads of its first group are issued before the routing so the latencies overlap
-  {
-    float v[4];
-    auto load = [&](int G0) {
+  unsigned long long* hseq = reinterpret_cast<unsigned long long*>(P.hdone + 2);
+  unsigned long long seq0 = 0;   // the counter at the start (producer lane 0)
+  if (tid == 0) seq0 = ld_relaxed_u64(hseq);
+  // the activations of K group warp - 1 (warps 1..17) are loaded before the routing and encoded
+  // as B-operand columns after it, while the producer already issues the weight copies
+  float xv[4] = {0.f, 0.f, 0.f, 0.f};
+  if (warp >= 1 && warp - 1 < nH)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) v[q] = bf16_bits_to_float(P.x[G0 * kGroup + q * 32 + lane]);
-    };
-    if (warp < nH) load(warp);
-    route_begin(s.rs, P, tid, kRThreads);
-    for (int G0 = warp; G0 < nH; G0 += kRWarps) {
-      if (G0 != warp) load(G0);
-      encode_group(v, xq + G0 * kGroup, xq + xcs + G0 * kGroup, reinterpret_cast<int4*>(xrec) + G0, lane);
-    }
-  }
+    for (int q = 0; q < 4; ++q) xv[q] = bf16_bits_to_float(P.x[(warp - 1) * kGroup + q * 32 + lane]);
+  route_begin(s.rs, P, tid, kRThreads);
   __syncthreads();
   route_finish(s.rs, P, tid, kRThreads);
+  if (tid < s.rs.nact) s.wsel[tid] = route_weight(s.rs, P, 0, s.rs.act[tid]);
+  __syncthreads();
   if (tid == 0) { trace_at(P, 1); trace_clk(P, 7); }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (warp >= 1) {
+    for (int G0 = warp - 1; G0 < nH; G0 += kRWarps - 1) {
+      if (G0 != warp - 1)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xv[q] = bf16_bits_to_float(P.x[G0 * kGroup + q * 32 + lane]);
+      encode_group(xv, xq + G0 * kGroup, xq + xcs + G0 * kGroup, reinterpret_cast<int4*>(xrec) + G0, lane);
+    }
+    tc::named_bar_sync(2, (kRWarps - 1) * 32);   // the columns are complete for warps 1..17
+  }
 
   const int G = gridDim.x, cta = blockIdx.x;
   RPlan pl;
@@ -160,11 +188,14 @@ __global__ void __launch_bounds__(kRThreads, 1)
       int okw = 1;
       if (lane == 0) {
         const long long t0 = clock64();
-        while (tc::ld_acquire(P.hdone) < G) {
+        const unsigned long long target = seq0 - seq0 % (unsigned long long)G + (unsigned long long)G;
+        while (ld_relaxed_u64(hseq) < target) {
           if (*abort || clock64() - t0 > tc::kWaitTimeoutCycles) { okw = 0; break; }
           __nanosleep(32);
         }
         if (okw) {
+          // acquire (pairs with the CTAs' release adds), then order the async-proxy copy after it
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");
           fence_proxy_async_global();
           trace_at(P, 4);
           trace_clk(P, 37);
@@ -293,12 +324,13 @@ __global__ void __launch_bounds__(kRThreads, 1)
       if (!ok) break;
       if (lane == 0) tc::mbar_arrive(&s.redfull[b]);
     }
-    // phase 2: 16 output rows over every selected expert; within a stage of eps experts, warp w
-    // takes expert w / (16 / eps) and one of 16 / eps equal parts of its 4 nI K chunks
+    // phase 2: 16 output rows over every selected expert. A stage holds ne <= eps experts' W2 rows,
+    // ne * nI K groups; warp w takes groups [w ne nI / 16, (w + 1) ne nI / 16). A group is four
+    // chunks = four h slices, each with its own scale a: the four MMAs run side by side and
+    // y += s * (sum_q a_q (256 D_hi + D_lo)_q - sum_q a_q 8 sum(v_q)).
     // (every compute warp runs the same block loop and meets the named barriers even after a
     // timeout; the waits then fail at once and the stores are skipped)
     if (pl.m > 0) {
-      const int P2 = kRCompute / pl.eps, el = w / P2, p2 = w % P2, cpp = 4 * nI / P2;
       bool h_in = false;
       for (int ob = cta; ob < nOB; ob += G) {
         float seg0 = 0.f, seg1 = 0.f;
@@ -310,41 +342,37 @@ __global__ void __launch_bounds__(kRThreads, 1)
             h_in = true;
             if (w == 0 && lane == 0) trace_clk(P, 40);
           }
-          if (el < min(pl.eps, pl.m - e0)) {
-            const int j = e0 + el;
-            const uint8_t* data = ring + (size_t)st * kRStage + el * 1024 * nI;
-            const uint16_t* scl = reinterpret_cast<const uint16_t*>(ring + (size_t)st * kRStage + kRData + el * sstride2);
-            const uint8_t* hs = hq + (size_t)j * nS * kSliceB;
-            // four chunks' MMAs are issued before the first result is used
-            for (int c0 = p2 * cpp; c0 < (p2 + 1) * cpp; c0 += 4) {
-              int d[4][4];
+          const int Gs = min(pl.eps, pl.m - e0) * nI;
+          const int gb = (w * Gs) >> 4, ge = ((w + 1) * Gs) >> 4;
+          int el = gb / nI, g2 = gb - el * nI;
+          for (int gl = gb; gl < ge; ++gl) {
+            const uint8_t* data = ring + (size_t)st * kRStage + el * 1024 * nI + g2 * 1024;
+            const uint16_t* scl =
+                reinterpret_cast<const uint16_t*>(ring + (size_t)st * kRStage + kRData + el * sstride2) + g2 * kORows;
+            const uint8_t* hs = hq + ((size_t)(e0 + el) * nS + 4 * g2) * kSliceB;
+            int d[4][4];
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int ci = c0 + q;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) d[q][e] = 0;
-                if (ci < (p2 + 1) * cpp) {
-                  const uint8_t* ch = data + ci * 256;
-                  const uint32_t wa = *reinterpret_cast<const uint32_t*>(ch + g * 16 + 4 * c);
-                  const uint32_t wb = *reinterpret_cast<const uint32_t*>(ch + (g + 8) * 16 + 4 * c);
-                  uint2 hb = make_uint2(0u, 0u);
-                  if (g < 2) hb = *reinterpret_cast<const uint2*>(hs + ci * kSliceB + g * 32 + c * 8);
-                  imma(d[q], wa & M, wb & M, (wa >> 4) & M, (wb >> 4) & M, hb.x, hb.y);
-                }
-              }
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const int ci = c0 + q;
-                if (ci < (p2 + 1) * cpp) {
-                  const int2 rec = *reinterpret_cast<const int2*>(hs + ci * kSliceB + 64);
-                  const float a = __int_as_float(rec.x);
-                  const float s0 = __uint_as_float((uint32_t)scl[(ci >> 2) * kORows + g] << 16);
-                  const float s1 = __uint_as_float((uint32_t)scl[(ci >> 2) * kORows + g + 8] << 16);
-                  seg0 = fmaf(s0 * a, (float)(d[q][0] * 256 + d[q][1] - rec.y), seg0);
-                  seg1 = fmaf(s1 * a, (float)(d[q][2] * 256 + d[q][3] - rec.y), seg1);
-                }
-              }
+            for (int q = 0; q < 4; ++q) {
+              const uint8_t* ch = data + q * 256;
+              const uint32_t wa = *reinterpret_cast<const uint32_t*>(ch + g * 16 + 4 * c);
+              const uint32_t wb = *reinterpret_cast<const uint32_t*>(ch + (g + 8) * 16 + 4 * c);
+              uint2 hb = make_uint2(0u, 0u);
+              if (g < 2) hb = *reinterpret_cast<const uint2*>(hs + q * kSliceB + g * 32 + c * 8);
+              imma0(d[q], wa & M, wb & M, (wa >> 4) & M, (wb >> 4) & M, hb.x, hb.y);
             }
+            const float s0 = __uint_as_float((uint32_t)scl[g] << 16);
+            const float s1 = __uint_as_float((uint32_t)scl[g + 8] << 16);
+            float t0 = 0.f, t1 = 0.f, cs = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 rec = *reinterpret_cast<const float2*>(hs + q * kSliceB + 64);   // {a, a * 8 sum v}
+              t0 = fmaf(rec.x, (float)(d[q][0] * 256 + d[q][1]), t0);
+              t1 = fmaf(rec.x, (float)(d[q][2] * 256 + d[q][3]), t1);
+              cs += rec.y;
+            }
+            seg0 = fmaf(s0, t0 - cs, seg0);
+            seg1 = fmaf(s1, t1 - cs, seg1);
+            if (++g2 == nI) { g2 = 0; ++el; }
           }
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&s.empty[st]);
@@ -385,8 +413,8 @@ __global__ void __launch_bounds__(kRThreads, 1)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.redempty[b]);
       const int j = u / nS, fs = u % nS;
-      const float wt = route_weight(s.rs, P, 0, s.rs.act[j]);
-      const float hv = (wt != 0.f) ? swiglu(gs, us) * wt : 0.f;
+      const float wt = s.wsel[j];
+      const float hv = (wt != 0.f) ? __fdividef(gs * us, 1.f + __expf(-gs)) * wt : 0.f;
       float mx = fabsf(hv);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
@@ -400,20 +428,30 @@ __global__ void __launch_bounds__(kRThreads, 1)
       const int at = (lane >> 3) * 8 + perm_pos(lane & 7);
       sl[at] = (uint8_t)h8;
       sl[32 + at] = (uint8_t)l8;
-      if (lane == 0) *reinterpret_cast<int2*>(sl + 64) = make_int2(__float_as_int(mx * (1.f / 32639.f)), 8 * sum);
+      if (lane == 0) {
+        const float a = mx * (1.f / 32639.f);
+        *reinterpret_cast<float2*>(sl + 64) = make_float2(a, a * (float)(8 * sum));
+      }
       if (lane == 0 && i < 4) trace_clk(P, 32 + i);
     }
-    fence_proxy_async_global();
     __syncwarp();   // the lanes' stores are ordered before lane 0's release
-    if (lane == 0 && ok && !*abort) tc::red_release_add(P.hdone, 1);
+    if (lane == 0 && ok && !*abort) red_release_add_u64(hseq, 1ull);
     if (lane == 0) trace_clk(P, 36);
     if (lane == 0) trace_at(P, 5);
   }
 
-  __syncthreads();
-  Plan fin{};
-  fin.n2 = pl.m;   // no expert selected: the outputs come from the accumulator alone
-  finish_launch(fin, P, abort, tid, kRThreads);
+  if (pl.m == 0 && !*abort) {   // no expert selected: the outputs come from the accumulator alone
+    for (int o = cta * kRThreads + tid; o < H; o += G * kRThreads) {
+      const float accv = P.accumulate ? __ldcg(P.acc + o) : 0.f;
+      if (P.out) {
+        P.out[o] = __bfloat16_as_ushort(__float2bfloat16_rn(accv));
+        if (P.accumulate) P.acc[o] = 0.f;
+      } else {
+        P.acc[o] = accv;
+      }
+    }
+  }
+  if (tid == 0) trace_at(P, 6);
 }
 
 // ---------------------------------------------------------------- host side
@@ -477,11 +515,11 @@ size_t rows_smem_bytes(int H, int I, int m_max) {
 }  // namespace
 
 // The single-token kernel takes H <= 2048 (a slice half's 32 rows x all K chunks fit one stage)
-// and I <= 2048 with I / 128 <= 8 or even (a stage holds 4 or 2 experts' 16-row W2 boxes).
+// and I <= 2048 (a stage holds 4 or 2 experts' 16-row W2 boxes).
 bool rows_supported(int T, int H, int I, int E, int k) {
   if (T != 1) return false;
   const int nH = H / kGroup, nI = I / kRowBlock;
-  if (nH < 1 || nH > 16 || nI < 1 || nI > 16 || (nI > 8 && (nI & 1))) return false;
+  if (nH < 1 || nH > 16 || nI < 1 || nI > 16) return false;
   return rows_smem_bytes(H, I, std::min(E, k)) <= (size_t)kSmemLimit;
 }
 
