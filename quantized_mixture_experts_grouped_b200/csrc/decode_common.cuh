@@ -144,16 +144,21 @@ __device__ inline void route_token_n(RouteSmem& rs, const DecParams& P, int t, i
   const float mx = logit_of(first);
   float el[8], sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 8; ++i) {   // rounds past k are skipped (a uniform branch)
+    el[i] = 0.f;
+    if (32 * i >= k) continue;
     const int j = 32 * i + lane;
-    el[i] = j < k ? expf(logit_of(mine[i]) - mx) : 0.f;
+    if (j < k) {
+      el[i] = expf(logit_of(mine[i]) - mx);
+      rs.idx[t * k + j] = 0xffff - (int)(mine[i] & 0xffffu);
+    }
     sum += el[i];
-    if (j < k) rs.idx[t * k + j] = 0xffff - (int)(mine[i] & 0xffffu);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    if (32 * i >= k) continue;
     const int j = 32 * i + lane;
     if (j < k) rs.wts[t * k + j] = el[i] / sum;
   }

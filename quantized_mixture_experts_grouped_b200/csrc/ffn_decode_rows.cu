@@ -88,6 +88,49 @@ __device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsig
   asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// Routing epilogue of the single token, one warp (k <= 32): from the k choices in rs.idx / rs.wts,
+// the selected resident experts in ascending id (rs.act, rs.sl, wsel; rank = set bits below the
+// expert in the presence mask), rs.nact, and the router outputs. A token routed twice to one
+// expert (given routing only) is reported and selects nothing.
+__device__ void route_one(RouteSmem& rs, float* wsel, const DecParams& P, int lane) {
+  const int k = P.k, E = P.E;
+  int e = -1;
+  float wv = 0.f;
+  if (lane < k) { e = rs.idx[lane]; wv = rs.wts[lane]; }
+  int sl = -1;
+  if (lane < k && (unsigned)e < (unsigned)E) sl = slot_of(P.slot, e);
+  const bool in = sl >= 0;
+  const int n_in = __popc(__ballot_sync(kFull, in));
+  const int nw = (E + 31) >> 5;
+  uint32_t mw = 0;   // lane wd < nw: presence word wd
+  for (int wd = 0; wd < nw; ++wd) {
+    const uint32_t v = __reduce_or_sync(kFull, (in && (e >> 5) == wd) ? 1u << (e & 31) : 0u);
+    if (lane == wd) mw = v;
+  }
+  int below = 0;
+  for (int wd = 0; wd < nw; ++wd) {
+    const uint32_t v = __shfl_sync(kFull, mw, wd);
+    if (in && wd < (e >> 5)) below += __popc(v);
+    if (in && wd == (e >> 5)) below += __popc(v & ((1u << (e & 31)) - 1u));
+  }
+  const int total = (int)__reduce_add_sync(kFull, (uint32_t)__popc(mw));
+  const bool dup = total != n_in;
+  if (in && !dup) {
+    rs.act[below] = e;
+    rs.sl[below] = sl;
+    wsel[below] = wv;
+  }
+  if (lane == 0) {
+    rs.nact = dup ? 0 : total;
+    rs.over = dup ? 1 : 0;
+    if (dup) report_status(P.ctl, MOE_ERR_ARG, kSiteOver);
+  }
+  if (P.logits && P.idx_out && blockIdx.x == 0 && lane < k) {
+    P.idx_out[lane] = e;
+    P.wts_out[lane] = wv;
+  }
+}
+
 // The split of both phases, identical in every CTA.
 struct RPlan {
   int m, nH, nI, nS;      // selected experts, K groups of H and I, slices per expert (I / 32)
@@ -122,6 +165,7 @@ __global__ void __launch_bounds__(kRThreads, 1)
   uint8_t* ring = hq + (ring_at - tc::smem_u32(hq));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  if (tid == 0) trace_clk(P, 60);
   if (warp == 0) {
     if (lane < kRStages) {
       tc::mbar_init(&s.full[lane], 1);
@@ -137,11 +181,11 @@ __global__ void __launch_bounds__(kRThreads, 1)
     }
     tc::fence_barrier_init();
   }
-  route_clear(s.rs, tid, kRThreads);
   __syncthreads();
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0) trace_at(P, 0);
+  if (tid == 0) trace_clk(P, 61);
   unsigned long long* hseq = reinterpret_cast<unsigned long long*>(P.hdone + 2);
   unsigned long long seq0 = 0;   // the counter at the start (producer lane 0)
   if (tid == 0) seq0 = ld_relaxed_u64(hseq);
@@ -151,10 +195,17 @@ __global__ void __launch_bounds__(kRThreads, 1)
   if (warp >= 1 && warp - 1 < nH)
 #pragma unroll
     for (int q = 0; q < 4; ++q) xv[q] = bf16_bits_to_float(P.x[(warp - 1) * kGroup + q * 32 + lane]);
-  route_begin(s.rs, P, tid, kRThreads);
-  __syncthreads();
-  route_finish(s.rs, P, tid, kRThreads);
-  if (tid < s.rs.nact) s.wsel[tid] = route_weight(s.rs, P, 0, s.rs.act[tid]);
+  if (warp == 0) {   // routing of the token and its grouping, one warp
+    if (P.logits) {
+      route_token(s.rs, P, 0, lane);
+    } else if (lane < P.k) {
+      s.rs.idx[lane] = P.idx_in[lane];
+      s.rs.wts[lane] = P.wts_in[lane];
+    }
+    __syncwarp();
+    if (tid == 0) trace_clk(P, 62);
+    route_one(s.rs, s.wsel, P, lane);
+  }
   __syncthreads();
   if (tid == 0) { trace_at(P, 1); trace_clk(P, 7); }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -517,7 +568,7 @@ size_t rows_smem_bytes(int H, int I, int m_max) {
 // The single-token kernel takes H <= 2048 (a slice half's 32 rows x all K chunks fit one stage)
 // and I <= 2048 (a stage holds 4 or 2 experts' 16-row W2 boxes).
 bool rows_supported(int T, int H, int I, int E, int k) {
-  if (T != 1) return false;
+  if (T != 1 || k > 32) return false;
   const int nH = H / kGroup, nI = I / kRowBlock;
   if (nH < 1 || nH > 16 || nI < 1 || nI > 16) return false;
   return rows_smem_bytes(H, I, std::min(E, k)) <= (size_t)kSmemLimit;
