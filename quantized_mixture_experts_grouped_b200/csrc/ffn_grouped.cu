@@ -130,6 +130,12 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile i
   return __all_sync(0xffffffffu, ok);
 }
 
+// Token-row maps of one operand with boxes of 128, 64 and 32 rows: a tile of at most 64 (32)
+// tokens loads only those rows, so its stages carry fewer bytes and turn over faster.
+struct alignas(64) BMaps {
+  CUtensorMap m[3];
+};
+
 struct TileDesc {
   int e, slot, chunk, bp, p0, ntok;
   size_t rb0, rb1;     // weight row blocks
@@ -153,7 +159,7 @@ __device__ __forceinline__ TileDesc describe(const GParams& P, int32_t packed) {
 }
 
 __global__ void __launch_bounds__(kGThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ CUtensorMap xmap) {
+grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ BMaps xm) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   // the dynamic shared window is only guaranteed 16-byte aligned: align the carve-out by hand
   GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
@@ -174,7 +180,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
     tc::mbar_init(&s.drain[1], 1);
     s.abort = 0;
     tc::fence_barrier_init();
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&xmap) : "memory");
+    for (int i = 0; i < 3; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.m[i]) : "memory");
   }
   if (warp == 1) {
     tc::tmem_alloc<kGTmemCols>(&s.tmem_base);
@@ -207,6 +213,9 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
       }
       if (stop) break;
       const TileDesc d = describe(P, P.tile_list[t]);
+      const int bi = d.ntok <= 32 ? 2 : (d.ntok <= 64 ? 1 : 0);   // token rows loaded: 128 >> bi
+      const CUtensorMap* xmap = &xm.m[bi];
+      const uint32_t bbytes = kBBoxBytes >> bi;
       const uint8_t* wb = P.w + (size_t)d.slot * P.w_stride;
       const uint16_t* sb = P.s + (size_t)d.slot * P.s_stride;
       bool ok = true;
@@ -215,9 +224,9 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ C
         if (!gwait(&s.empty[st], ((it / kGStages) & 1) ^ 1, abort)) { ok = false; break; }
         if (lane == 0) {
           GStage& S = s.st[st];
-          tc::mbar_arrive_expect_tx(&s.full[st], 2 * kBBoxBytes + 2 * 8192 + 2 * 256);
-          tma_load_2d(S.b[0], &xmap, g * 128, d.p0, &s.full[st]);
-          tma_load_2d(S.b[1], &xmap, g * 128 + 64, d.p0, &s.full[st]);
+          tc::mbar_arrive_expect_tx(&s.full[st], 2 * bbytes + 2 * 8192 + 2 * 256);
+          tma_load_2d(S.b[0], xmap, g * 128, d.p0, &s.full[st]);
+          tma_load_2d(S.b[1], xmap, g * 128 + 64, d.p0, &s.full[st]);
           const size_t t0 = d.rb0 * P.G + g, t1 = d.rb1 * P.G + g;
           tc::bulk_g2s(S.w[0], wb + t0 * kTileBytes, 8192, &s.full[st], pol_w);
           tc::bulk_g2s(S.w[1], wb + t1 * kTileBytes, 8192, &s.full[st], pol_w);
@@ -525,12 +534,12 @@ int get_encode() {
   return MOE_OK;
 }
 
-// 2-D map over a row-major bf16 matrix [rows][cols]: box = 64 columns x 128 rows, 128B swizzle.
-int make_rows_map(CUtensorMap* map, const void* base, int rows, int cols) {
+// 2-D map over a row-major bf16 matrix [rows][cols]: box = 64 columns x box_rows rows, 128B swizzle.
+int make_rows_map(CUtensorMap* map, const void* base, int rows, int cols, int box_rows) {
   if (int rc = get_encode()) return rc;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kTokTile};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -550,7 +559,7 @@ int sm_count() {
   return g_sms;
 }
 
-int launch_gemm(const GParams& P, const CUtensorMap& map, int max_tiles, cudaStream_t s) {
+int launch_gemm(const GParams& P, const BMaps& map, int max_tiles, cudaStream_t s) {
   const size_t smem = sizeof(GSmem) + 1024;
   static bool attr = false;
   if (!attr) {
@@ -611,9 +620,11 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
     return rc;
   const int max_chunks = (Tk + kTokTile - 1) / kTokTile + a.E;
 
-  CUtensorMap xmap, hmap;
-  if (int rc = make_rows_map(&xmap, xp, Tk, a.H)) return rc;
-  if (int rc = make_rows_map(&hmap, hp, Tk, a.I)) return rc;
+  BMaps xmap, hmap;
+  for (int i = 0; i < 3; ++i) {
+    if (int rc = make_rows_map(&xmap.m[i], xp, Tk, a.H, kTokTile >> i)) return rc;
+    if (int rc = make_rows_map(&hmap.m[i], hp, Tk, a.I, kTokTile >> i)) return rc;
+  }
 
   GParams P{};
   P.w = a.w13; P.s = a.s13;
