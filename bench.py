@@ -552,15 +552,46 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
     idx = torch.empty((T, k), dtype=torch.int32, device=device)
     wts = torch.empty((T, k), dtype=torch.float32, device=device)
     out = torch.empty((T, H), dtype=torch.bfloat16, device=device)
-    out_host = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
     ws = q.alloc_workspace(T, H, I, E, k, device)
+    # end to end: two buffer sets (inputs on the device, outputs on the device and in pinned host
+    # memory), step i uses set i % 2; copies on two copy streams overlap the neighbouring steps
+    xs2 = [torch.empty_like(x) for _ in range(2)]
+    lgs2 = [torch.empty_like(lg) for _ in range(2)]
+    outs2 = [torch.empty_like(out) for _ in range(2)]
+    out_host = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     flags = q.PATHS[args.path]
     s = torch.cuda.Stream(device)
     peaks, peaks_kind = load_peaks()
     sampler = ClockSampler(local)
 
-    def call(xx, ll):
-        q.moe_w4a16_layer(xx, ll, k, w13, s13, w2, s2, H, I, idx, wts, ws, out, flags=flags, stream=s)
+    def call(xx, ll, oo=out):
+        q.moe_w4a16_layer(xx, ll, k, w13, s13, w2, s2, H, I, idx, wts, ws, oo, flags=flags, stream=s)
+
+    h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_ready = [torch.cuda.Event(), torch.cuda.Event()]
+    computed = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    pending = [None]
+
+    def e2e_step(i):
+        """Inputs up (copy stream), the layer, the output back (second copy stream); the host
+        waits for the previous step's output, one step behind."""
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            h2d.wait_event(done[b])            # step i - 2 is computed and copied out of set b
+            xs2[b].copy_(x_host, non_blocking=True)
+            lgs2[b].copy_(lg_host, non_blocking=True)
+            in_ready[b].record(h2d)
+        s.wait_event(in_ready[b])
+        call(xs2[b], lgs2[b], outs2[b])
+        computed[b].record(s)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(computed[b])
+            out_host[b].copy_(outs2[b], non_blocking=True)
+            done[b].record(d2h)
+        if pending[0] is not None:
+            done[pending[0]].synchronize()
+        pending[0] = b
 
     with torch.cuda.stream(s):
         n0 = q.moe_launch_count()
@@ -586,20 +617,18 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
         clocks = sampler.stop()
         ms = all_max(e0.elapsed_time(e1), world) / args.steps
         # end to end: inputs from pinned host memory, output back to the host, every step
-        for _ in range(args.warmup):
-            x.copy_(x_host, non_blocking=True); lg.copy_(lg_host, non_blocking=True)
-            call(x, lg)
-            out_host.copy_(out, non_blocking=True)
+        for i in range(args.warmup):
+            e2e_step(i)
+        done[pending[0]].synchronize()
+        pending[0] = None
         s.synchronize()
         barrier(world)
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(s)
-        for _ in range(args.steps):
-            x.copy_(x_host, non_blocking=True); lg.copy_(lg_host, non_blocking=True)
-            call(x, lg)
-            out_host.copy_(out, non_blocking=True)
-            s.synchronize()
-        f1.record(s)
+        h2d.wait_event(f0)                     # the first timed input copy starts after f0
+        for i in range(args.steps):
+            e2e_step(args.warmup + i)
+        f1.record(d2h)                         # after the last step's output is in host memory
         f1.synchronize()
         e2e_ms = all_max(f0.elapsed_time(f1), world) / args.steps
     status = q.moe_workspace_status(ws, s)
