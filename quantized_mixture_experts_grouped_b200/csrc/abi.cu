@@ -50,7 +50,7 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
   L.tiles = take(sizeof(int32_t) * (4 * (E + 1) + 64));
   {
     const size_t chunks = (Tk + 127) / 128 + (size_t)E;
-    const size_t blocks = std::max<size_t>(I / 128, H / 256 + 1);
+    const size_t blocks = std::max<size_t>(I / 128, H / 128);   // gate/up pairs; down pairs x K halves
     L.tile_list_len = chunks * blocks;
     L.tile_list = take(sizeof(int32_t) * 2 * L.tile_list_len);
   }

@@ -17,6 +17,11 @@
 // Tile list: per expert, ceil(n_e / 128) token chunks x row-block pairs; MMA N is the chunk's
 // token count rounded up to 16, so a ragged tail costs at most 15 padded tokens per expert.
 // Tiles are claimed dynamically (atomic counter). Every wait is bounded.
+// Split K for the down GEMM: when the down tiles would fill the SMs only about once (few token
+// chunks, long K = I), each tile's K range is split in two halves that run as separate tiles and
+// write separate bf16 partial outputs; the combine adds the two partials of each row (in a fixed
+// order) before applying the router weight. This fills the second round of SMs with half-length
+// tiles instead of leaving most of them idle while a few full-length tiles finish.
 #include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -70,6 +75,8 @@ struct GParams {
   int G;                                    // K / 128
   int rows_half;                            // gate/up: I (up block offset); down: unused
   int mode;
+  int ksplit;                               // down: K halves per tile (1 or 2); gate/up: 1
+  size_t part_stride;                       // elements between the partial outputs of the K halves
   const int32_t* tile_list;                 // packed tiles
   const int32_t* ntiles;                    // total tile count (device)
   const int32_t* offsets;                   // grouped pair offsets [E+1]
@@ -138,12 +145,30 @@ struct alignas(64) BMaps {
 
 struct TileDesc {
   int e, slot, chunk, bp, p0, ntok;
+  int g0, g1;          // K groups [g0, g1) of this tile
+  int part;            // K half (index of the partial output)
   size_t rb0, rb1;     // weight row blocks
 };
+
+// K range of a tile: the whole K, or one of two halves when K is split (the block-pair field
+// then holds pair * 2 + half)
+__device__ __forceinline__ void k_range(const GParams& P, int& bp, int& g0, int& g1, int& part) {
+  if (P.ksplit == 2) {
+    part = bp & 1;
+    bp >>= 1;
+    g0 = part ? P.G / 2 : 0;
+    g1 = part ? P.G : P.G / 2;
+  } else {
+    part = 0;
+    g0 = 0;
+    g1 = P.G;
+  }
+}
 
 __device__ __forceinline__ TileDesc describe(const GParams& P, int32_t packed) {
   TileDesc d;
   unpack_tile(packed, d.e, d.chunk, d.bp);
+  k_range(P, d.bp, d.g0, d.g1, d.part);
   d.slot = slot_of(P.table, d.e);
   const int n_e = P.offsets[d.e + 1] - P.offsets[d.e];
   d.p0 = P.offsets[d.e] + d.chunk * kTokTile;
@@ -219,7 +244,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
       const uint8_t* wb = P.w + (size_t)d.slot * P.w_stride;
       const uint16_t* sb = P.s + (size_t)d.slot * P.s_stride;
       bool ok = true;
-      for (int g = 0; g < P.G; ++g, ++it) {
+      for (int g = d.g0; g < d.g1; ++g, ++it) {
         const int st = it % kGStages;
         if (!gwait(&s.empty[st], ((it / kGStages) & 1) ^ 1, abort)) { ok = false; break; }
         if (lane == 0) {
@@ -270,7 +295,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
         tc::tc_fence_after();
         if (me == 0 && n == 1) gtrace(P, 3);
         bool ok = true;
-        for (int g = 0; g < P.G; ++g, ++it, ++a_it) {
+        for (int g = d.g0; g < d.g1; ++g, ++it, ++a_it) {
           const int st = it % kGStages, ab = a_it & 1;
           if (!tc::mbar_wait(&s.full[st], (it / kGStages) & 1, abort) ||
               !tc::mbar_wait(&s.afull[ab], (a_it >> 1) & 1, abort)) {
@@ -284,7 +309,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t baddr = bbase + (kk >> 2) * kBBoxBytes + (kk & 3) * 32;
             const uint64_t bdesc = tc::smem_desc(baddr, 16, 1024, 2);
-            tc::mma_ts(dacc, a + kk * 8, bdesc, idesc, (g > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_ts(dacc, a + kk * 8, bdesc, idesc, (g > d.g0 || kk > 0) ? 1u : 0u);
           }
           tc::mma_commit(&s.aempty[ab]);
           tc::mma_commit(&s.empty[st]);
@@ -316,8 +341,10 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.tq_empty[q]);
       if (packed < 0) break;
+      int bp = packed & 0xfff, g0, g1, part;
+      k_range(P, bp, g0, g1, part);
       bool ok = true;
-      for (int g = 0; g < P.G; ++g, ++it, ++a_it) {
+      for (int g = g0; g < g1; ++g, ++it, ++a_it) {
         const int st = it % kGStages, ab = a_it & 1;
         if (!gwait(&s.full[st], (it / kGStages) & 1, abort)) { ok = false; break; }
         const uint8_t* wsrc = s.st[st].w[blk];
@@ -416,8 +443,10 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           }
         }
       } else {
-        // 256 columns = 32 pieces per token row; a warp stores one whole row per step
+        // 256 columns = 32 pieces per token row; a warp stores one whole row per step (into the
+        // partial output of the tile's K half)
         const size_t col = d.rb0 * kRowBlock + (etid & 31) * 8;
+        uint16_t* const outp = P.out + (size_t)d.part * P.part_stride;
         for (int t0 = 0; t0 < d.ntok; t0 += 16) {
           uint4 v[4];
 #pragma unroll
@@ -425,7 +454,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
 #pragma unroll
           for (int m = 0; m < 4; ++m) {
             const int t = t0 + (etid >> 5) + 4 * m;
-            if (t < d.ntok) *reinterpret_cast<uint4*>(P.out + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
+            if (t < d.ntok) *reinterpret_cast<uint4*>(outp + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
           }
         }
       }
@@ -476,8 +505,8 @@ __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t* __restric
 }
 
 // out[t] = bf16( acc + sum_j wts[t][j] * y[inv[t][j]] ) over the bf16 down-projection rows y,
-// in fixed j order.
-__global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __restrict__ yw,
+// in fixed j order. With K split in two, y = y_0 + y_1 (the halves' partial rows, added first).
+__global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __restrict__ yw, size_t part_stride,
                                                            const float* __restrict__ wts,
                                                            const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ inv,
@@ -495,13 +524,26 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __res
   for (int j = 0; j < k; ++j) {
     if (slot_of(table, idx[(size_t)t * k + j]) < 0) continue;
     const float w = wts[(size_t)t * k + j];
-    const uint4 y = *reinterpret_cast<const uint4*>(yw + (size_t)inv[(size_t)t * k + j] * H + n0);
+    const uint16_t* yrow = yw + (size_t)inv[(size_t)t * k + j] * H + n0;
+    const uint4 y = *reinterpret_cast<const uint4*>(yrow);
     const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
+    float yf[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] = fmaf(w, bf16_bits_to_float(yy[i] & 0xffffu), v[2 * i]);
-      v[2 * i + 1] = fmaf(w, bf16_bits_to_float(yy[i] >> 16), v[2 * i + 1]);
+      yf[2 * i] = bf16_bits_to_float(yy[i] & 0xffffu);
+      yf[2 * i + 1] = bf16_bits_to_float(yy[i] >> 16);
     }
+    if (part_stride) {
+      const uint4 z = *reinterpret_cast<const uint4*>(yrow + part_stride);
+      const uint32_t zz[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        yf[2 * i] += bf16_bits_to_float(zz[i] & 0xffffu);
+        yf[2 * i + 1] += bf16_bits_to_float(zz[i] >> 16);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(w, yf[i], v[i]);
   }
   if (out) {
     uint32_t pk[4];
@@ -587,6 +629,7 @@ int launch_gemm(const GParams& P, const BMaps& map, int max_tiles, cudaStream_t 
 
 bool ffn_grouped_supported(const FfnArgs& a) {
   return a.T >= 1 && a.E <= kMaxExperts && a.H % 256 == 0 && a.I % kRowBlock == 0 && (size_t)a.T * a.k < (1u << 20) &&
+         a.H / kRowBlock < 4096 && a.I / kRowBlock < 4096 &&   // 12-bit block field of a packed tile
          (a.T * a.k + kTokTile - 1) / kTokTile < 4096;
 }
 
@@ -602,7 +645,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   int32_t* list_dn = list_gu + L.tile_list_len;
   uint16_t* xp = reinterpret_cast<uint16_t*>(a.ws + L.xp);
   uint16_t* hp = reinterpret_cast<uint16_t*>(a.ws + L.hp);
-  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // y per pair, bf16
+  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // y per pair, bf16 (one or two K-half partials)
   int* ctl = reinterpret_cast<int*>(a.ws + L.status);
 
   if (int rc = launch_permute(a.idx, a.T, a.k, a.E, counts, offsets, perm, inv,
@@ -610,13 +653,17 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
     return rc;
   if (int rc = launch_gather_rows(a.x, perm, Tk, a.k, a.H, xp, s)) return rc;
   const int IB = a.I / kRowBlock, HP = a.H / 256;
+  // K split of the down GEMM: two halves when even the fewest token chunks this batch can have
+  // give fewer than two rounds of down tiles on the SMs, and K holds at least two groups
+  const int min_chunks = (Tk + kTokTile - 1) / kTokTile;
+  const int ksplit = (a.I / kGroup >= 2 && (long long)min_chunks * HP < 2LL * sm_count()) ? 2 : 1;
   note_launch();
   if (int rc = check_cuda(launch_pdl(tile_list_kernel, dim3(a.E), dim3(256), 0, s, (const int32_t*)counts, a.E, a.slot,
                                      IB, list_gu, tiles + 0), "tile_list_kernel"))
     return rc;
   note_launch();
   if (int rc = check_cuda(launch_pdl(tile_list_kernel, dim3(a.E), dim3(256), 0, s, (const int32_t*)counts, a.E, a.slot,
-                                     HP, list_dn, tiles + 1), "tile_list_kernel"))
+                                     HP * ksplit, list_dn, tiles + 1), "tile_list_kernel"))
     return rc;
   const int max_chunks = (Tk + kTokTile - 1) / kTokTile + a.E;
 
@@ -630,6 +677,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   P.w = a.w13; P.s = a.s13;
   P.w_stride = (size_t)2 * a.I * a.H / 2; P.s_stride = (size_t)2 * a.I * (a.H / kGroup);
   P.K = a.H; P.G = a.H / kGroup; P.rows_half = a.I; P.mode = kModeGateUp;
+  P.ksplit = 1; P.part_stride = 0;
   P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
   P.perm = perm; P.wts = a.wts; P.out = hp; P.out_ld = a.I; P.Tk = Tk; P.ctl = ctl;
   P.trace = nullptr;
@@ -638,13 +686,14 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   P.w = a.w2; P.s = a.s2;
   P.w_stride = (size_t)a.H * a.I / 2; P.s_stride = (size_t)a.H * (a.I / kGroup);
   P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
+  P.ksplit = ksplit; P.part_stride = ksplit == 2 ? (size_t)Tk * a.H : 0;   // the partials fill the fp32-sized yp
   P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;
   P.trace = dec::g_trace;
-  if (int rc = launch_gemm(P, hmap, max_chunks * HP, s)) return rc;
+  if (int rc = launch_gemm(P, hmap, max_chunks * HP * ksplit, s)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
   note_launch();
-  return check_cuda(launch_pdl(combine_bf16_kernel, grid, dim3(256), 0, s, (const uint16_t*)yw, a.wts, a.idx,
+  return check_cuda(launch_pdl(combine_bf16_kernel, grid, dim3(256), 0, s, (const uint16_t*)yw, P.part_stride, a.wts, a.idx,
                                (const int32_t*)inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
                                a.accumulate, a.out),
                     "combine_bf16_kernel");
