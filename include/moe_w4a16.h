@@ -129,7 +129,9 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  *   y_e(x) = W2_e . ( silu(W_gate_e . x) * (W_up_e . x) ),  silu(z) = z / (1 + exp(-z))
  *   out[t] = sum_{j<k} wts[t][j] * y_{idx[t][j]}(x_t)
  * with W = q * s dequantised from the packed banks. The tcgen05 paths multiply bf16 operands
- * (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the default fused decode kernel
+ * (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the grouped path rounds each
+ * token-expert pair's down projection to bf16 (when it splits K in two, each half, the halves
+ * then added in fp32) before the router-weighted combine; the default fused decode kernel
  * (T <= 16) multiplies the codes exactly with x and h held as 16-bit fixed point per
  * 128-element group (32 for h at T = 1; error <= max|group| / 65278), scales applied in fp32.
  * out is bf16.
