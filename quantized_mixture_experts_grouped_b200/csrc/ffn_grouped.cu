@@ -3,7 +3,7 @@
 // through fused grouped MoE kernels).
 //
 // Launch sequence: permute (group pairs by expert) -> gather rows -> tile plan -> gate/up GEMM
-// with fused silu(g)*u -> down GEMM with the router weight fused in its epilogue -> combine.
+// with fused silu(g)*u -> down GEMM (bf16 rows per token-expert pair) -> router-weighted combine.
 //
 // Both GEMMs are one persistent tcgen05 kernel (sm_100a). A CTA tile is a PAIR of 128-row
 // weight blocks (gate rows f..f+127 and the matching up rows, or two consecutive row blocks of
@@ -83,8 +83,8 @@ struct GParams {
   const int32_t* table;                     // expert -> slot (nullable)
   unsigned long long* trace;                // optional per-CTA clock stamps (diagnostics)
   const int32_t* perm;                      // pair id of grouped position
-  const float* wts;                         // router weights [T*k]
-  uint16_t* out;                            // gate/up: Hp [Tk][I]; down: Yp [Tk][H] (weighted)
+  const float* wts;                         // router weights [T*k] (applied by the combine)
+  uint16_t* out;                            // gate/up: Hp [Tk][I]; down: Yp [Tk][H] (unweighted)
   int out_ld;                               // row length of out
   int Tk;
   int* ctl;
