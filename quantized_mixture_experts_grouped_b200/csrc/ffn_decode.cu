@@ -3,6 +3,11 @@
 // Memory-Efficient W4A16 Inference", Abstract: all selected experts execute through fused
 // grouped MoE kernels; the router's top-k is unchanged).
 //
+// This file holds the path's dispatch (ffn_decode: the single-token kernel of
+// ffn_decode_rows.cu at T = 1, the warp-MMA kernel of ffn_decode_mma.cu up to 16 tokens) and the
+// tcgen05 variant of the fused launch described below, which runs on request
+// (MOE_PATH_DECODE_TC) as the bf16 tensor-core comparison point.
+//
 // A decode batch (T <= 16 tokens) reads every selected expert's packed weights exactly once, so
 // the layer is bound by HBM bandwidth on those bytes plus the latency of its dependent steps.
 // On B200 a CTA only streams near its share of HBM bandwidth when it moves weights in large
