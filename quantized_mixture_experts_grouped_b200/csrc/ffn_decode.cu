@@ -69,7 +69,6 @@ constexpr int kABufs = 4;                  // dequantised tiles in tensor memory
 constexpr int kIssuers = 2;                // MMA-issuing threads (one per warp)
 constexpr int kAcc = 8;                    // accumulators per issuer (16 columns each)
 constexpr int kThreads = 480;              // 15 warps
-constexpr int kWarps = kThreads / 32;
 constexpr int kIssuerWarp0 = 1;
 constexpr int kEpiWarp0 = 2;               // warps 2..5
 constexpr int kDqWarp0 = 6;                // warps 6..13: two groups of four
