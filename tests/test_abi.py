@@ -75,3 +75,17 @@ def test_argument_errors_before_launch():
     h = ctypes.c_void_p(0)
     rc = L.moe_slot_cache_create(8, 2, 256, 128, p, p, p, p, None, p, p, p, ctypes.byref(h))
     assert rc == q.MOE_ERR_ARG and not h.value
+
+
+def test_binding_constants_match_the_header():
+    """The Python binding's status, path and flag constants are the header's enum values."""
+    import quantized_mixture_experts_grouped_b200 as q
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    values = {n: int(v, 0) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(0x[0-9a-fA-F]+|\d+)", text)}
+    for name in ("MOE_OK", "MOE_ERR_ARG", "MOE_ERR_SHAPE", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
+                 "MOE_PATH_AUTO", "MOE_PATH_SIMPLE", "MOE_PATH_DECODE", "MOE_PATH_GROUPED",
+                 "MOE_PATH_SEQUENTIAL", "MOE_PATH_DECODE_TC", "MOE_FLAG_ACCUMULATE"):
+        assert values[name] == getattr(q, name), name
+    assert sorted(q.PATHS.values()) == sorted(values[n] for n in values if n.startswith("MOE_PATH_")
+                                              and n != "MOE_PATH_MASK")
+    assert q.lib.moe_packed_layout_version() == 1
