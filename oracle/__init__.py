@@ -1,7 +1,7 @@
 """Plain CPU oracle of the fused grouped W4A16 MoE FFN layer (ctypes wrapper).
 
 TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU-baseline leg
-are the only callers. The product library never imports this package, and this package
+and reference arm (``bench.py --impl reference``) are the only callers. The product library never imports this package, and this package
 imports nothing from the product package. The arithmetic lives in ``oracle.cpp`` (plain
 C++17 loops); this module only compiles it with g++ and marshals numpy arrays.
 

@@ -1,8 +1,8 @@
 // Plain CPU oracle for the fused grouped W4A16 mixture-of-experts FFN layer.
 //
 // TEST INFRASTRUCTURE ONLY. This file is the slow, obviously-correct definition that the CUDA
-// path is checked against. Only the tests, the smoke check and the CPU-baseline leg of the
-// benchmark may load it; the product library never links, loads or calls it, and this file
+// path is checked against. Only the tests, the smoke check and the benchmark's CPU-baseline leg
+// and reference arm may load it; the product library never links, loads or calls it, and this file
 // includes nothing from the product tree.
 //
 // Source of the method: "Every Expert Counts: ExactMoE for Memory-Efficient W4A16 Inference"
