@@ -89,3 +89,37 @@ def test_binding_constants_match_the_header():
     assert sorted(q.PATHS.values()) == sorted(values[n] for n in values if n.startswith("MOE_PATH_")
                                               and n != "MOE_PATH_MASK")
     assert q.lib.moe_packed_layout_version() == 1
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """The header compiles as C99 and a C program linked against the library calls its host-side
+    entry points (sizes, versions, argument errors: nothing that touches a device)."""
+    import shutil
+    import subprocess
+    import quantized_mixture_experts_grouped_b200 as q
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "moe_w4a16.h"
+int main(void) {
+  size_t ws = 0;
+  if (moe_abi_version() != 1 || moe_packed_layout_version() != 1) return 1;
+  if (moe_packed_bytes(2048, 2048) != (size_t)2048 * 2048 / 2) return 2;
+  if (moe_scales_count(2048, 1024) != (size_t)2048 * 8) return 3;
+  if (moe_workspace_bytes(1, 2048, 1024, 64, 8, &ws) != MOE_OK || ws == 0) return 4;
+  if (moe_workspace_bytes(1, 2000, 1024, 64, 8, &ws) != MOE_ERR_SHAPE) return 5;
+  if (moe_quantize_pack(NULL, 1, 128, 128, NULL, NULL, NULL) != MOE_ERR_ARG) return 6;
+  if (moe_last_error_string() == NULL) return 7;
+  printf("ok %zu\n", ws);
+  return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    lib_dir = os.path.dirname(q.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                           "-o", str(exe), "-L", lib_dir, "-l:libmoe_w4a16.so", f"-Wl,-rpath,{lib_dir}"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, (out.returncode, out.stdout, out.stderr)
+    assert out.stdout.startswith("ok ")
