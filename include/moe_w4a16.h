@@ -202,7 +202,8 @@ typedef struct moe_slot_cache moe_slot_cache;
 /* bank_* are HOST pointers to pinned memory (cudaHostAlloc / torch pin_memory) holding all E
  * experts in expert order; pool_* are device pointers with room for S experts in slot order.
  * Both stay owned by the caller and must outlive the cache. The cache starts empty.
- * *out receives a host-allocated handle. Errors: MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA. */
+ * *out receives a host-allocated handle. Creating the cache makes no CUDA call (the events of
+ * moe_slot_cache_layer are created on its first call). Errors: MOE_ERR_ARG, MOE_ERR_SHAPE. */
 int moe_slot_cache_create(int E, int S, int H, int I,
                           const uint8_t* bank_w13, const uint16_t* bank_s13,
                           const uint8_t* bank_w2, const uint16_t* bank_s2,
@@ -217,8 +218,10 @@ void moe_slot_cache_destroy(moe_slot_cache* cache);
  * expert; misses (HOST, int32 [S]) and *n_misses receive the experts loaded, in load order.
  * The copies wait for `reuse_ok` (an event recorded after the last kernel that read the pool;
  * may be NULL) and are issued on copy_stream; `loaded` (may be NULL) is recorded on
- * copy_stream after them. A failed copy leaves the cache state unchanged and returns
- * MOE_ERR_CUDA. */
+ * copy_stream after them. A failed copy returns MOE_ERR_CUDA with nothing of the wave
+ * committed: needed_mask, the LRU clock and times are unchanged and no table is written; the
+ * slots this wave had already started to overwrite are marked free (their contents are no
+ * longer the experts they held). */
 int slot_table_update(moe_slot_cache* cache, uint64_t* needed_mask,
                       int32_t* wave_table, int32_t* misses, int* n_misses,
                       moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded);
@@ -226,6 +229,11 @@ int slot_table_update(moe_slot_cache* cache, uint64_t* needed_mask,
 /* Testing aid for failure handling: the n-th next refill copy of this cache (0 = the next
  * one) reports failure as if cudaMemcpyAsync had returned an error; n = -1 turns it off. */
 void moe_slot_cache_fail_copy_after(moe_slot_cache* cache, int n);
+
+/* Testing aid for the replacement policy: with dry != 0, slot_table_update plans and commits
+ * every wave as usual but issues no copy (bank and pool are never touched), so the policy runs
+ * on a machine without a GPU; dry = 0 restores the copies. */
+void moe_slot_cache_dry_run(moe_slot_cache* cache, int dry);
 
 /* Host view of the cache state: slot_expert[S] (-1 free), last_used[S]; returns the clock. */
 int64_t moe_slot_cache_state(const moe_slot_cache* cache, int32_t* slot_expert, int64_t* last_used);

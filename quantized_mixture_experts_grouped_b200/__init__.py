@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "moe_slot_cache_create": ([I, I, I, I, P, P, P, P, P, P, P, P, c.POINTER(P)], I),
         "moe_slot_cache_destroy": ([P], None),
         "moe_slot_cache_fail_copy_after": ([P, I], None),
+        "moe_slot_cache_dry_run": ([P, I], None),
         "slot_table_update": ([P, P, P, P, c.POINTER(I), P, P, P], I),
         "moe_slot_cache_state": ([P, P, P], c.c_int64),
         "moe_slot_cache_layer": ([P, P, P, I, I, P, P, P, P, Z, P, I, P, P, c.POINTER(I), c.POINTER(I)], I),
@@ -191,6 +192,10 @@ class SlotCache:
 
     def fail_copy_after(self, n: int):
         lib.moe_slot_cache_fail_copy_after(self.handle, n)
+
+    def dry_run(self, dry: bool = True):
+        """Plan and commit refills without copying (testing the policy without a GPU)."""
+        lib.moe_slot_cache_dry_run(self.handle, int(dry))
 
     def state(self):
         import numpy as np

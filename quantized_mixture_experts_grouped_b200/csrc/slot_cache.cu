@@ -27,6 +27,7 @@ struct moe_slot_cache {
   std::vector<int32_t> wave_tables;                  // host copies of every wave's table
   std::vector<int32_t> idx_host;
   int fail_copies_after = -1;                        // test hook: fail the n-th next copy
+  bool dry_run = false;                              // test hook: plan and commit, copy nothing
 };
 
 namespace moe {
@@ -37,6 +38,12 @@ MOE_API void moe_slot_cache_fail_copy_after(moe_slot_cache* c, int n) {
   if (c) c->fail_copies_after = n;
 }
 
+// Test hook: with dry != 0 refills are planned and committed exactly as usual but no copy is
+// issued, so the replacement policy runs on a machine without a GPU; 0 restores the copies.
+MOE_API void moe_slot_cache_dry_run(moe_slot_cache* c, int dry) {
+  if (c) c->dry_run = dry != 0;
+}
+
 namespace {
 
 cudaError_t refill_copy(moe_slot_cache* c, void* dst, const void* src, size_t bytes, cudaStream_t s) {
@@ -45,7 +52,20 @@ cudaError_t refill_copy(moe_slot_cache* c, void* dst, const void* src, size_t by
     return cudaErrorInvalidValue;
   }
   if (c->fail_copies_after > 0) c->fail_copies_after--;
+  if (c->dry_run) return cudaSuccess;
   return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, s);
+}
+
+// The events that order refills against the FFN launches of moe_slot_cache_layer, created on
+// its first call (creating the cache itself makes no CUDA call).
+int ensure_events(moe_slot_cache* c) {
+  if (!c->compute_done)
+    if (int rc = check_cuda(cudaEventCreateWithFlags(&c->compute_done, cudaEventDisableTiming), "event create"))
+      return rc;
+  if (!c->loaded)
+    if (int rc = check_cuda(cudaEventCreateWithFlags(&c->loaded, cudaEventDisableTiming), "event create"))
+      return rc;
+  return MOE_OK;
 }
 
 }  // namespace
@@ -74,15 +94,6 @@ MOE_API int moe_slot_cache_create(int E, int S, int H, int I, const uint8_t* ban
   c->slot_expert.assign(S, -1);
   c->last_used.assign(S, 0);
   c->wave_tables.assign((size_t)E * (E + 1), -1);
-  if (int rc = check_cuda(cudaEventCreateWithFlags(&c->compute_done, cudaEventDisableTiming), "event create")) {
-    delete c;
-    return rc;
-  }
-  if (int rc = check_cuda(cudaEventCreateWithFlags(&c->loaded, cudaEventDisableTiming), "event create")) {
-    cudaEventDestroy(c->compute_done);
-    delete c;
-    return rc;
-  }
   *out = c;
   return MOE_OK;
 }
@@ -190,6 +201,7 @@ MOE_API int moe_slot_cache_layer(moe_slot_cache* c, const uint16_t* x, const uin
   *n_waves = 0;
   *n_loads = 0;
   if (T == 0) return MOE_OK;
+  if (int rc = ensure_events(c)) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int E = c->E;
   if (int rc = moe_route_topk(logits, T, E, k, idx, wts, stream)) return rc;
