@@ -100,7 +100,7 @@ def quantize(w_bf16: np.ndarray):
 
 
 def pack(q: np.ndarray, s: np.ndarray):
-    """q int8 [N][K], s uint16 [N][K/128] -> (packed uint8 [N*K/2], scales uint16 tiled [N*K/128])."""
+    """q int8 [N][K], s uint16 [N][K/128] -> (packed uint8 [N*K/2], scales uint16 in the packed order [N*K/128])."""
     q = np.ascontiguousarray(q, dtype=np.int8)
     s = np.ascontiguousarray(s, dtype=np.uint16)
     N, K = q.shape
@@ -110,18 +110,18 @@ def pack(q: np.ndarray, s: np.ndarray):
     return packed, st
 
 
-def unpack(packed: np.ndarray, scales_tiled: np.ndarray, N: int, K: int):
+def unpack(packed: np.ndarray, scales_packed: np.ndarray, N: int, K: int):
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
-    st = np.ascontiguousarray(scales_tiled, dtype=np.uint16)
+    st = np.ascontiguousarray(scales_packed, dtype=np.uint16)
     q = np.zeros((N, K), np.int8)
     s = np.zeros((N, K // 128), np.uint16)
     _check(lib().orc_unpack(_p(packed), _p(st), N, K, _p(q), _p(s)), "unpack")
     return q, s
 
 
-def dequant(packed: np.ndarray, scales_tiled: np.ndarray, N: int, K: int) -> np.ndarray:
+def dequant(packed: np.ndarray, scales_packed: np.ndarray, N: int, K: int) -> np.ndarray:
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
-    st = np.ascontiguousarray(scales_tiled, dtype=np.uint16)
+    st = np.ascontiguousarray(scales_packed, dtype=np.uint16)
     out = np.zeros((N, K), np.float32)
     _check(lib().orc_dequant(_p(packed), _p(st), N, K, _p(out)), "dequant")
     return out

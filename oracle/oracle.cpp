@@ -33,8 +33,9 @@
 namespace {
 
 constexpr int kGroup = 128;          // quantisation group along K (the abstract's "group-128")
-constexpr int kRowBlock = 128;       // rows per packed tile
-constexpr int kTileBytes = kRowBlock * kGroup / 2;   // 8192 bytes of codes per tile
+constexpr int kRowBlock = 128;       // N must be a multiple of this (the kernels' row blocks)
+constexpr int kRowGroup = 8;         // rows per packed chunk
+constexpr int kChunkBytes = kRowGroup * kGroup / 2;   // 512 bytes of codes per chunk
 
 float bf16_to_f32(uint16_t b) {
   uint32_t u = (uint32_t)b << 16;
@@ -53,18 +54,19 @@ uint16_t f32_to_bf16(float f) {
   return (uint16_t)(u >> 16);
 }
 
-// ---- packed layout index map (layout "MW4T v1", our own design) ----
-// A matrix W[N][K] (N, K multiples of 128) is cut into tiles of 128 rows x 128 K (one
-// quantisation group per row per tile). Tiles are stored row-block-major: tile (rb, g) at
-// byte (rb*G + g) * 8192, G = K/128. Inside a tile, the 128 K values of a row are split into
-// four quarters of 32; quarter kq of row r is a 16-byte chunk at kq*2048 + r*16. Inside the
-// chunk, K values 8w..8w+7 form little-endian 32-bit word w; element e of that word
+// ---- packed layout index map (layout "MW4T v2", our own design) ----
+// A matrix W[N][K] (N, K multiples of 128) is cut into row groups of 8 rows (R = n/8) and K
+// groups of 128 (g = k/128, the quantisation groups; G = K/128). The codes of row group R and K
+// group g are one 512-byte chunk at byte (R*G + g) * 512, so the chunks of one row group over
+// all of K follow each other. Inside a chunk, the 128 K values of a row are split into four
+// quarters of 32; quarter kq of row r8 = n%8 is the 16-byte piece at kq*128 + r8*16. Inside the
+// piece, K values 8w..8w+7 form little-endian 32-bit word w; element e of that word
 // (e = 2p + h) sits in the nibble at bit 16*h + 4*p. Each nibble holds the offset-binary code
 // c = q + 8, so every byte holds two codes.
 size_t code_offset(int N, int K, int n, int k, int* shift) {
   (void)N;
   const int G = K / kGroup;
-  const int rb = n / kRowBlock, r = n % kRowBlock;
+  const int R = n / kRowGroup, r8 = n % kRowGroup;
   const int g = k / kGroup, kk = k % kGroup;
   const int kq = kk / 32;
   const int w = (kk % 32) / 8;
@@ -72,13 +74,13 @@ size_t code_offset(int N, int K, int n, int k, int* shift) {
   const int p = e / 2, h = e % 2;
   const int bit = 16 * h + 4 * p;
   *shift = bit % 8;
-  return ((size_t)rb * G + g) * kTileBytes + (size_t)kq * 2048 + (size_t)r * 16 + (size_t)w * 4 + bit / 8;
+  return ((size_t)R * G + g) * kChunkBytes + (size_t)kq * 128 + (size_t)r8 * 16 + (size_t)w * 4 + bit / 8;
 }
 
-// Scales are stored tile-major as well: scale(n, g) at ((rb*G + g)*128 + r).
+// Scales follow the same chunk order: scale(n, g) at ((R*G + g)*8 + r8).
 size_t scale_index(int K, int n, int g) {
   const int G = K / kGroup;
-  return ((size_t)(n / kRowBlock) * G + g) * kRowBlock + (n % kRowBlock);
+  return ((size_t)(n / kRowGroup) * G + g) * kRowGroup + (n % kRowGroup);
 }
 
 int code_at(const uint8_t* packed, int N, int K, int n, int k) {
@@ -142,10 +144,10 @@ int orc_quantize(const uint16_t* w, int N, int K, int8_t* q, uint16_t* s) {
   return 0;
 }
 
-// Packs q[N][K] (values -8..7) and row-major scales s[N][K/128] into the tiled layout
+// Packs q[N][K] (values -8..7) and row-major scales s[N][K/128] into the chunked layout
 // described at code_offset() / scale_index().
-int orc_pack(const int8_t* q, const uint16_t* s, int N, int K, uint8_t* packed, uint16_t* scales_tiled) {
-  if (!q || !s || !packed || !scales_tiled || !shape_ok(N, K)) return 1;
+int orc_pack(const int8_t* q, const uint16_t* s, int N, int K, uint8_t* packed, uint16_t* scales_packed) {
+  if (!q || !s || !packed || !scales_packed || !shape_ok(N, K)) return 1;
   const int G = K / kGroup;
   std::memset(packed, 0, orc_packed_bytes(N, K));
   for (int n = 0; n < N; ++n)
@@ -157,26 +159,26 @@ int orc_pack(const int8_t* q, const uint16_t* s, int N, int K, uint8_t* packed, 
       packed[off] |= (uint8_t)((qv + 8) << sh);
     }
   for (int n = 0; n < N; ++n)
-    for (int g = 0; g < G; ++g) scales_tiled[scale_index(K, n, g)] = s[(size_t)n * G + g];
+    for (int g = 0; g < G; ++g) scales_packed[scale_index(K, n, g)] = s[(size_t)n * G + g];
   return 0;
 }
 
 // Inverse of orc_pack: recovers q[N][K] and row-major scales s[N][K/128].
-int orc_unpack(const uint8_t* packed, const uint16_t* scales_tiled, int N, int K, int8_t* q, uint16_t* s) {
-  if (!packed || !scales_tiled || !q || !s || !shape_ok(N, K)) return 1;
+int orc_unpack(const uint8_t* packed, const uint16_t* scales_packed, int N, int K, int8_t* q, uint16_t* s) {
+  if (!packed || !scales_packed || !q || !s || !shape_ok(N, K)) return 1;
   const int G = K / kGroup;
   for (int n = 0; n < N; ++n)
     for (int k = 0; k < K; ++k) q[(size_t)n * K + k] = (int8_t)(code_at(packed, N, K, n, k) - 8);
   for (int n = 0; n < N; ++n)
-    for (int g = 0; g < G; ++g) s[(size_t)n * G + g] = scales_tiled[scale_index(K, n, g)];
+    for (int g = 0; g < G; ++g) s[(size_t)n * G + g] = scales_packed[scale_index(K, n, g)];
   return 0;
 }
 
 // Dequantises a packed matrix to fp32: out[N][K] = q * s (exact).
-int orc_dequant(const uint8_t* packed, const uint16_t* scales_tiled, int N, int K, float* out) {
-  if (!packed || !scales_tiled || !out || !shape_ok(N, K)) return 1;
+int orc_dequant(const uint8_t* packed, const uint16_t* scales_packed, int N, int K, float* out) {
+  if (!packed || !scales_packed || !out || !shape_ok(N, K)) return 1;
   for (int n = 0; n < N; ++n)
-    for (int k = 0; k < K; ++k) out[(size_t)n * K + k] = (float)weight_at(packed, scales_tiled, N, K, n, k);
+    for (int k = 0; k < K; ++k) out[(size_t)n * K + k] = (float)weight_at(packed, scales_packed, N, K, n, k);
   return 0;
 }
 
