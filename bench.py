@@ -54,27 +54,32 @@ def expert_bytes(H: int, I: int) -> int:
     return codes + scales
 
 
-PROFILE = os.path.join(ROOT, "profiles", "moe_decode_rows_kernel_olmoe_decode.md")
+PROFILE = os.path.join(ROOT, "profiles", "moe_decode_rows_kernel_olmoe_decode.json")
 PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_rows.cu",
-                   "quantized_mixture_experts_grouped_b200/csrc/decode_common.cuh"]
+                   "quantized_mixture_experts_grouped_b200/csrc/decode_common.cuh",
+                   "quantized_mixture_experts_grouped_b200/csrc/common.cuh",
+                   "quantized_mixture_experts_grouped_b200/csrc/tc.cuh"]
+
+
+def source_hash(files=None) -> str:
+    """First 16 hex digits of the SHA-256 of the profiled kernel's source files, in order."""
+    import hashlib
+    files = PROFILE_SOURCES if files is None else files
+    return hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in files)).hexdigest()[:16]
 
 
 def profiled_traffic():
-    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu summary,
-    or None when the summary is missing or the kernel's sources changed since the capture."""
-    import hashlib
-    import re
+    """DRAM bytes (read + write) per launch of the decode kernel from the committed ncu record
+    (profiles/*.json: "source_hash", "traffic_bytes_per_launch"), or None when the record is
+    missing or the kernel's sources changed since the capture."""
     try:
-        text = open(PROFILE).read()
-        digest = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read()
-                                         for f in PROFILE_SOURCES)).hexdigest()[:16]
-    except OSError:
+        rec = json.load(open(PROFILE))
+        digest = source_hash()
+    except (OSError, ValueError):
         return None
-    m_hash = re.search(r"kernel source hash \([^)]*\): ([0-9a-f]+)", text)
-    m_tr = re.search(r"traffic_bytes_per_launch: ([0-9]+)", text)
-    if not m_hash or not m_tr or m_hash.group(1) != digest:
+    if rec.get("source_hash") != digest or not isinstance(rec.get("traffic_bytes_per_launch"), int):
         return None
-    return int(m_tr.group(1))
+    return rec["traffic_bytes_per_launch"]
 
 
 def load_peaks():
@@ -524,13 +529,31 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         bench.e2e_drain()
         e2e_ms = all_max(f0.elapsed_time(f1), world)
     status = bench.q.moe_workspace_status(bench.ws, s)
+    distinct_mean = bench.distinct_experts_mean()
+    h2d_bytes, d2h_bytes = bench.h2d_bytes(), bench.d2h_bytes()
 
+    launches_per_layer = bench.launches_per_step / wl.layers
+    del bench
+    torch.cuda.empty_cache()
+    # the prefill layer measured in the same process (a figure for the tensor-bound side)
+    secondary = None
+    if not args.no_secondary and wl.name == "olmoe_decode":
+        pw = mi.WORKLOADS["olmoe_prefill"]
+        r = measure_single_layer(pw, "auto", 20, 3, world, local)
+        secondary = {"workload": pw.name, "us_per_layer": r["ms"] * 1e3, "tokens_per_s": pw.T * world / (r["ms"] / 1e3),
+                     "e2e_tokens_per_s": pw.T * world / (r["e2e_ms"] / 1e3),
+                     "achieved_tflops": r["achieved"], "peak_tflops": r["peak"], "frac": r["achieved"] / r["peak"],
+                     "peak_kind": f"{r['peaks_kind']} bf16 dense (burst)", "steps": 20, "warmup": 3,
+                     "clocks": r["clocks"], "device_status": r["status"]}
     if rank != 0:
         return
     tokens = wl.T * args.steps * world
     value = tokens / (ms_total / 1e3)
-    bytes_per_layer = bench.distinct_experts_mean() * expert_bytes(wl.H, wl.I)
-    achieved = bytes_per_layer / (layer_ms / 1e3) / 1e9
+    bytes_per_layer = distinct_mean * expert_bytes(wl.H, wl.I)
+    # duration of the one launch of a layer: the timed step over its layers (the launches of a
+    # step run back to back, so this includes the gap between two launches)
+    us_layer = ms_total / args.steps / wl.layers * 1e3
+    achieved = bytes_per_layer / (us_layer / 1e6) / 1e9
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -540,18 +563,21 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak,
                      "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
-                     "kernel": ("moe_decode_kernel" if args.path == "decode_tc" else
-                                ("moe_decode_rows_kernel" if wl.T == 1 else "moe_decode_mma_kernel"))
-                               + " (the one launch per layer; event pair per layer)"
-                               if args.path in ("auto", "decode", "decode_tc") else "all launches of the layer (event pair per layer)",
-                     "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": layer_ms * 1e3,
+                     "kernel": ("moe_decode_rows_kernel" if wl.T == 1 else "moe_decode_mma_kernel")
+                               + " (the one launch per layer; duration = timed step / layers)"
+                               if args.path in ("auto", "decode") else "all launches of the layer (timed step / layers)",
+                     "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": us_layer,
+                     "launches_per_layer": launches_per_layer,
+                     "us_per_launch_event_pair": layer_ms * 1e3,
                      "peak_kind": f"{peaks_kind} HBM copy"},
-        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": bench.h2d_bytes(),
-                "d2h_bytes_per_step": bench.d2h_bytes()},
-        "gpu_launches": bench.launches_per_step * args.steps,
+        "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": d2h_bytes},
+        "gpu_launches": int(launches_per_layer * wl.layers) * args.steps,
         "clocks": clocks,
         "device_status": status,
     }
+    if secondary is not None:
+        line["secondary"] = secondary
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
@@ -582,9 +608,10 @@ def cpu_baseline_tokens(wl: mi.Workload, budget_s: float = 12.0):
                       f"work, experts packed by the oracle)"}
 
 
-def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
+def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, world: int, local: int) -> dict:
     """Large-batch workloads (prefill, large expert): one layer of T tokens per step through
-    moe_w4a16_layer (route, permute, gather, two grouped GEMMs, combine)."""
+    moe_w4a16_layer (route, permute, gather, two grouped GEMMs, combine), timed with CUDA events
+    (max over ranks) with inputs resident, then end to end with host copies every step."""
     import quantized_mixture_experts_grouped_b200 as q
     device = torch.device("cuda", local)
     H, I, E, k, T = wl.H, wl.I, wl.E, wl.k, wl.T
@@ -607,7 +634,7 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
     lgs2 = [torch.empty_like(lg) for _ in range(2)]
     outs2 = [torch.empty_like(out) for _ in range(2)]
     out_host = [torch.empty((T, H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    flags = q.PATHS[args.path]
+    flags = q.PATHS[path]
     s = torch.cuda.Stream(device)
     peaks, peaks_kind = load_peaks()
     sampler = ClockSampler(local)
@@ -645,7 +672,7 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
         n0 = q.moe_launch_count()
         call(x, lg)
         launches = q.moe_launch_count() - n0
-        for _ in range(args.warmup):
+        for _ in range(warmup):
             call(x, lg)
         s.synchronize()
         sampler.start()
@@ -657,15 +684,15 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
-        for _ in range(args.steps):
+        for _ in range(steps):
             call(x, lg)
         e1.record(s)
         e1.synchronize()
         barrier(world)
         clocks = sampler.stop()
-        ms = all_max(e0.elapsed_time(e1), world) / args.steps
+        ms = all_max(e0.elapsed_time(e1), world) / steps
         # end to end: inputs from pinned host memory, output back to the host, every step
-        for i in range(args.warmup):
+        for i in range(warmup):
             e2e_step(i)
         done[pending[0]].synchronize()
         pending[0] = None
@@ -674,17 +701,27 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(s)
         h2d.wait_event(f0)                     # the first timed input copy starts after f0
-        for i in range(args.steps):
-            e2e_step(args.warmup + i)
+        for i in range(steps):
+            e2e_step(warmup + i)
         f1.record(d2h)                         # after the last step's output is in host memory
         f1.synchronize()
-        e2e_ms = all_max(f0.elapsed_time(f1), world) / args.steps
+        e2e_ms = all_max(f0.elapsed_time(f1), world) / steps
     status = q.moe_workspace_status(ws, s)
-    if rank != 0:
-        return
     flops = 6.0 * H * I * T * k
     achieved = flops / (ms / 1e3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    res = dict(ms=ms, e2e_ms=e2e_ms, clocks=clocks, status=status, launches=launches, achieved=achieved,
+               peak=peak, peaks_kind=peaks_kind, h2d=(x.numel() + lg.numel()) * 2, d2h=out.numel() * 2)
+    del w13, s13, w2, s2, ws, xs2, lgs2, outs2
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
+    r = measure_single_layer(wl, args.path, args.steps, args.warmup, world, local)
+    if rank != 0:
+        return
+    T, ms, e2e_ms, achieved, peak = wl.T, r["ms"], r["e2e_ms"], r["achieved"], r["peak"]
     line = {
         "metric": METRIC, "value": T * world / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -695,12 +732,12 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
                      "frac": achieved / peak, "traffic": None,
                      "kernel": "whole layer (route, permute, gather, gate/up and down grouped GEMMs, combine): "
                                "6*H*I*T*k flop over the layer's event-timed duration",
-                     "peak_kind": f"{peaks_kind} bf16 dense (burst)"},
+                     "peak_kind": f"{r['peaks_kind']} bf16 dense (burst)"},
         "e2e": {"value": T * world / (e2e_ms / 1e3), "unit": "tokens/s",
-                "h2d_bytes_per_step": (x.numel() + lg.numel()) * 2, "d2h_bytes_per_step": out.numel() * 2},
-        "gpu_launches": launches * args.steps,
-        "clocks": clocks,
-        "device_status": status,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": r["clocks"],
+        "device_status": r["status"],
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_tokens(wl)
@@ -826,8 +863,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="olmoe_decode",
                     choices=["olmoe_decode", "olmoe_slots", "olmoe_prefill", "large_expert"])
-    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "decode_tc", "grouped", "sequential"])
+    ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped", "sequential"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the prefill layer measured after the default decode workload")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers than the workload's (profiling runs only; the metric uses 16)")
     ap.add_argument("--tokens", type=int, default=None,

@@ -18,14 +18,15 @@
  *  - Calls are asynchronous on the given stream (a cudaStream_t; NULL = legacy default
  *    stream) and return a status: MOE_OK, or an error whose text moe_last_error_string()
  *    gives. Argument errors are reported before anything is launched.
- *  - Packed weight layout "MW4T v1" (this library's own design; the abstract stores experts
- *    in a kernel-native form without giving its bytes): a matrix W[N][K] is cut into tiles of
- *    128 rows x 128 K, stored row-block-major (tile (rb, g) at byte (rb*K/128 + g)*8192).
- *    Inside a tile, quarter kq (32 K values) of row r is a 16-byte chunk at kq*2048 + r*16;
- *    K values 8w..8w+7 of the chunk form little-endian 32-bit word w, element 2p+h sitting in
- *    the nibble at bit 16h+4p. A nibble holds the offset-binary code q+8, two codes per byte.
- *    Scales are bf16, one per (row, group of 128 K), stored tile-major: scale(n, g) at
- *    ((n/128)*(K/128) + g)*128 + n%128.
+ *  - Packed weight layout "MW4T v2" (this library's own design; the abstract stores experts
+ *    in a kernel-native form without giving its bytes): a matrix W[N][K] is cut into chunks of
+ *    8 rows x 128 K (one quantisation group of each of the 8 rows), 512 bytes each; the chunk
+ *    of row group R = n/8 and K group g is at byte (R*K/128 + g)*512, so the chunks of one row
+ *    group follow each other over all of K. Inside a chunk, quarter kq (32 K values) of row
+ *    r8 = n%8 is a 16-byte piece at kq*128 + r8*16; K values 8w..8w+7 of the piece form
+ *    little-endian 32-bit word w, element 2p+h sitting in the nibble at bit 16h+4p. A nibble
+ *    holds the offset-binary code q+8, two codes per byte. Scales are bf16, one per (row,
+ *    group of 128 K), in the same chunk order: scale(n, g) at ((n/8)*(K/128) + g)*8 + n%8.
  */
 #ifndef MOE_W4A16_H
 #define MOE_W4A16_H
@@ -56,13 +57,12 @@ enum {
                               int8 warp-MMA path, in-kernel combine                          */
   MOE_PATH_GROUPED = 3,    /* permute + tcgen05 grouped GEMMs (gate/up, down) + combine       */
   MOE_PATH_SEQUENTIAL = 4, /* one expert at a time through the same kernels (ablation)        */
-  MOE_PATH_DECODE_TC = 5,  /* the fused launch with bf16 tcgen05 MMAs (T <= 16; comparison)   */
   MOE_PATH_MASK = 0xff,
   MOE_FLAG_ACCUMULATE = 0x100 /* add this call's contribution into the workspace fp32
                                  accumulator instead of starting from zero (slot-cache waves) */
 };
 
-/* Version of this ABI and of the packed layout ("MW4T v1" -> 1). */
+/* Version of this ABI and of the packed layout ("MW4T v2" -> 2). */
 int moe_abi_version(void);
 int moe_packed_layout_version(void);
 
@@ -77,6 +77,14 @@ unsigned long long moe_launch_count(void);
  * timestamps (%globaltimer, 64 unsigned 64-bit slots per CTA, one row per CTA) into it; NULL
  * turns recording off. The buffer must hold 64 * (number of SMs) slots. */
 void moe_debug_set_decode_trace(void* dev_buffer);
+
+/* Testing aid for failure detection (process-wide; for tests only). `cycles` > 0 sets the limit,
+ * in SM clock cycles, of the bounded waits of the single-token decode kernel (0 restores the
+ * default of about two seconds). `extra_arrivals` > 0 makes that kernel's exchange between CTAs
+ * wait for that many arrivals more than it launches: the wait cannot be satisfied, runs out, the
+ * kernel records MOE_ERR_TIMEOUT in the workspace status word and exits without writing its
+ * outputs. 0 turns it off. */
+void moe_debug_set_wait_limit(unsigned long long cycles, int extra_arrivals);
 
 /* Bytes of packed codes of one N x K matrix (N*K/2) and number of its bf16 scales
  * (N*K/128). Return 0 when N or K is not a positive multiple of 128. */
@@ -114,8 +122,11 @@ int moe_permute(const int32_t* idx, int T, int k, int E,
 
 /* Workspace of moe_w4a16_ffn / moe_w4a16_layer for these sizes (device memory, 256-byte
  * aligned, owned by the caller). It must be zeroed once with moe_workspace_init before its
- * first use; the kernels leave their counters zeroed again when they finish. One workspace
- * must not be used by two calls that can run at the same time. */
+ * first use; the kernels leave their counters zeroed again when they finish. A workspace sized
+ * for T tokens serves calls with any T' <= T (any path) on the same H, I and E: the words that
+ * must start at zero sit at offsets that depend on H, I and E only. Zero it again with
+ * moe_workspace_init when H, I or E change, and after moe_workspace_status has reported a
+ * failure. One workspace must not be used by two calls that can run at the same time. */
 int moe_workspace_bytes(int T, int H, int I, int E, int k, size_t* bytes);
 int moe_workspace_init(void* workspace, size_t bytes, moe_stream_t stream);
 
@@ -140,11 +151,12 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  *     slot stride = moe_packed_bytes / moe_scales_count of the matrix.
  *   slot_of_expert: int32 [E] device table, expert -> slot; NULL = identity (slot e holds
  *     expert e). An entry of -1 skips that expert's pairs (a later slot-cache wave runs them).
- *   workspace: see moe_workspace_bytes. out: bf16 [T][H], or NULL with MOE_FLAG_ACCUMULATE
- *     to only add into the fp32 accumulator (a non-final slot-cache wave).
+ *   workspace: see moe_workspace_bytes. out: bf16 [T][H], or NULL to leave this call's sum in
+ *     the workspace's fp32 accumulator (a non-final slot-cache wave).
  * flags: a MOE_PATH_* value, optionally | MOE_FLAG_ACCUMULATE. Without ACCUMULATE the
- * accumulator starts from zero; with it, earlier waves' sums are included. The fp32
- * accumulator is zeroed again after out is written.
+ * accumulator is not read: this call's sum replaces it (out NULL) or is the output. With
+ * ACCUMULATE, the sums of earlier waves in the accumulator are added. The fp32 accumulator is
+ * zeroed again after out is written with ACCUMULATE.
  * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA (launch failure). */
 int moe_w4a16_ffn(const uint16_t* x_bf16, int T, int H, int I, int E, int k,
                   const int32_t* idx, const float* wts,
@@ -176,8 +188,9 @@ int moe_w4a16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16,
  *    current); make that first call before any stream capture on the device.
  *  - Every call on a device shares the array: calls that can run at the same time (other
  *    streams, other host threads) race, so the caller must serialise them.
- *  - Each call clears, on `stream`, the parts that must start at zero (status/control block
- *    and the fused-decode counters). Device-side failures are not reported by this entry.
+ *  - Each call clears, on `stream`, the parts that must start at zero (control block and the
+ *    fused-decode counters). A device-side failure (a bounded wait that ran out) is kept in the
+ *    array's status word until moe_noalloc_status reads it.
  *  - Nothing is allocated.
  * Errors: MOE_ERR_SHAPE when these sizes need more than the array holds (use moe_w4a16_layer
  * with a caller workspace), MOE_ERR_ARG for MOE_FLAG_ACCUMULATE (the fp32 accumulator would be
@@ -189,6 +202,11 @@ int moe_w4a16_layer_noalloc(const uint16_t* x_bf16, const uint16_t* logits_bf16,
                             const int32_t* slot_of_expert,
                             int32_t* idx, float* wts,
                             uint16_t* out_bf16, int flags, moe_stream_t stream);
+
+/* Reads (synchronously, on `stream`) and clears the status word of the array that
+ * moe_w4a16_layer_noalloc uses on the current device: 0 when every call since the last read
+ * finished normally on the device, else the MOE_ERR_* code of the first failure. */
+int moe_noalloc_status(moe_stream_t stream, int* status);
 
 /* ---- GPU slot cache (abstract: "configurable GPU-resident slot cache", experts kept in
  * pinned host memory). One cache per layer: S device slots, each holding one expert's packed

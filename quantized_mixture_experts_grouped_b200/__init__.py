@@ -19,10 +19,9 @@ LIB_PATH = os.path.join(_HERE, "libmoe_w4a16.so")
 
 MOE_OK, MOE_ERR_ARG, MOE_ERR_SHAPE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = 0, 1, 2, 3, 4
 MOE_PATH_AUTO, MOE_PATH_SIMPLE, MOE_PATH_DECODE, MOE_PATH_GROUPED, MOE_PATH_SEQUENTIAL = 0, 1, 2, 3, 4
-MOE_PATH_DECODE_TC = 5
 MOE_FLAG_ACCUMULATE = 0x100
 PATHS = {"auto": MOE_PATH_AUTO, "simple": MOE_PATH_SIMPLE, "decode": MOE_PATH_DECODE,
-         "grouped": MOE_PATH_GROUPED, "sequential": MOE_PATH_SEQUENTIAL, "decode_tc": MOE_PATH_DECODE_TC}
+         "grouped": MOE_PATH_GROUPED, "sequential": MOE_PATH_SEQUENTIAL}
 
 
 class MoeError(RuntimeError):
@@ -44,6 +43,7 @@ def _load() -> ctypes.CDLL:
         "moe_last_error_string": ([], c.c_char_p),
         "moe_launch_count": ([], c.c_ulonglong),
         "moe_debug_set_decode_trace": ([P], None),
+        "moe_debug_set_wait_limit": ([c.c_ulonglong, I], None),
         "moe_packed_bytes": ([I, I], Z),
         "moe_scales_count": ([I, I], Z),
         "moe_quantize_pack": ([P, I, I, I, P, P, P], I),
@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "moe_w4a16_ffn": ([P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P, I, P], I),
         "moe_w4a16_layer": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P, I, P], I),
         "moe_w4a16_layer_noalloc": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, I, P], I),
+        "moe_noalloc_status": ([P, c.POINTER(I)], I),
         "moe_slot_cache_create": ([I, I, I, I, P, P, P, P, P, P, P, P, c.POINTER(P)], I),
         "moe_slot_cache_destroy": ([P], None),
         "moe_slot_cache_fail_copy_after": ([P, I], None),
@@ -99,6 +100,12 @@ def moe_abi_version() -> int:
 
 def moe_launch_count() -> int:
     return lib.moe_launch_count()
+
+
+def moe_debug_set_wait_limit(cycles: int, extra_arrivals: int = 0):
+    """Testing aid: bounded-wait limit of the single-token decode kernel (0 = default) and extra
+    arrivals its exchange waits for (> 0 makes that wait run out)."""
+    lib.moe_debug_set_wait_limit(cycles, extra_arrivals)
 
 
 def moe_packed_bytes(N: int, K: int) -> int:
@@ -166,6 +173,13 @@ def moe_w4a16_layer_noalloc(x, logits, k: int, w13, s13, w2, s2, H: int, I: int,
     T, E = logits.shape
     _err(lib.moe_w4a16_layer_noalloc(_p(x), _p(logits), T, H, I, E, k, _p(w13), _p(s13), _p(w2), _p(s2),
                                      _p(slot_of_expert), _p(idx), _p(wts), _p(out), flags, _s(stream)))
+
+
+def moe_noalloc_status(stream=None) -> int:
+    """Reads and clears the device status word of the static array of moe_w4a16_layer_noalloc."""
+    st = ctypes.c_int(0)
+    _err(lib.moe_noalloc_status(_s(stream), ctypes.byref(st)))
+    return st.value
 
 
 class SlotCache:

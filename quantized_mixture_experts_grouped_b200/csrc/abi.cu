@@ -42,6 +42,7 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
     return at;
   };
   L.status = take(sizeof(int32_t) * kCtlWords);
+  L.ctr = take(decode_counter_bytes(H, I, E));
   L.counts = take(sizeof(int32_t) * E);
   L.offsets = take(sizeof(int32_t) * (E + 1));
   L.perm = take(sizeof(int32_t) * Tk);
@@ -79,10 +80,8 @@ int check_layer_args(const uint16_t* x, int T, int H, int I, int E, int k, const
   if (!dims_ok(H, I)) return fail(MOE_ERR_SHAPE, "H=%d and I=%d must be positive multiples of 128", H, I);
   if (!w13 || !s13 || !w2 || !s2 || !ws) return fail(MOE_ERR_ARG, "null weight or workspace pointer");
   if (T > 0 && !x) return fail(MOE_ERR_ARG, "null x");
-  if (!out && !(flags & MOE_FLAG_ACCUMULATE) && T > 0)
-    return fail(MOE_ERR_ARG, "out may be NULL only with MOE_FLAG_ACCUMULATE");
   const int path = flags & MOE_PATH_MASK;
-  if (path > MOE_PATH_DECODE_TC) return fail(MOE_ERR_ARG, "unknown path %d", path);
+  if (path > MOE_PATH_SEQUENTIAL) return fail(MOE_ERR_ARG, "unknown path %d", path);
   const WsLayout L = ws_layout(T, H, I, E, k);
   if (ws_bytes < L.total)
     return fail(MOE_ERR_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, L.total);
@@ -104,7 +103,6 @@ int run_ffn(const FfnArgs& a, int flags, cudaStream_t s) {
     case MOE_PATH_SEQUENTIAL:
       return ffn_sequential(a, s);
     case MOE_PATH_DECODE:
-    case MOE_PATH_DECODE_TC:
       if (!ffn_decode_supported(a)) return fail(MOE_ERR_SHAPE, "fused decode path does not support these sizes");
       return ffn_decode(a, s);
     case MOE_PATH_GROUPED:
@@ -120,7 +118,7 @@ int run_ffn(const FfnArgs& a, int flags, cudaStream_t s) {
 }  // namespace
 
 MOE_API int moe_abi_version(void) { return 1; }
-MOE_API int moe_packed_layout_version(void) { return 1; }
+MOE_API int moe_packed_layout_version(void) { return 2; }
 MOE_API const char* moe_last_error_string(void) { return g_last_error.c_str(); }
 MOE_API unsigned long long moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
@@ -209,7 +207,6 @@ MOE_API int moe_w4a16_ffn(const uint16_t* x_bf16, int T, int H, int I, int E, in
   a.idx = idx; a.wts = wts; a.w13 = w13; a.s13 = s13; a.w2 = w2; a.s2 = s2;
   a.slot = slot_of_expert; a.ws = static_cast<char*>(workspace); a.ws_bytes = workspace_bytes;
   a.out = out_bf16; a.accumulate = (flags & MOE_FLAG_ACCUMULATE) != 0;
-  a.tc_decode = (flags & MOE_PATH_MASK) == MOE_PATH_DECODE_TC;
   return run_ffn(a, flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -228,9 +225,8 @@ MOE_API int moe_w4a16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16,
   a.slot = slot_of_expert; a.ws = static_cast<char*>(workspace); a.ws_bytes = workspace_bytes;
   a.out = out_bf16; a.accumulate = (flags & MOE_FLAG_ACCUMULATE) != 0;
   const int path = flags & MOE_PATH_MASK;
-  a.tc_decode = path == MOE_PATH_DECODE_TC;
   const bool fused =
-      (path == MOE_PATH_DECODE || path == MOE_PATH_DECODE_TC || path == MOE_PATH_AUTO) && ffn_decode_supported(a);
+      (path == MOE_PATH_DECODE || path == MOE_PATH_AUTO) && ffn_decode_supported(a);
   if (fused) {
     a.logits = logits_bf16; a.idx_out = idx; a.wts_out = wts;
     return ffn_decode(a, s);

@@ -13,9 +13,22 @@
 namespace moe {
 
 constexpr int kGroup = 128;        // quantisation group along K
-constexpr int kRowBlock = 128;     // rows per packed tile
+constexpr int kRowBlock = 128;     // rows per kernel tile (N is a multiple of it)
 constexpr int kTileBytes = 8192;   // codes of one 128 x 128 tile
+constexpr int kRowGroup = 8;       // rows per packed chunk
+constexpr int kChunkBytes = 512;   // codes of one chunk: 8 rows x 128 K
 constexpr int kMaxExperts = 256;
+
+// Packed layout "MW4T v2" of a matrix W[N][K] (see include/moe_w4a16.h): byte offset of the
+// 512-byte chunk of row group R = n / 8 and K group g, and index of its first scale.
+__host__ __device__ __forceinline__ size_t chunk_offset(int R, int g, int G) {
+  return ((size_t)R * G + g) * kChunkBytes;
+}
+__host__ __device__ __forceinline__ size_t chunk_scale_index(int R, int g, int G) {
+  return ((size_t)R * G + g) * kRowGroup;
+}
+// Inside a chunk: the 16-byte piece of quarter kq (32 K values) of row r8 (0..7).
+__host__ __device__ __forceinline__ int piece_offset(int kq, int r8) { return kq * 128 + r8 * 16; }
 
 // ---- host-side error reporting (thread-local text, see moe_last_error_string) ----
 int fail(int code, const char* fmt, ...);
@@ -32,6 +45,8 @@ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 // ---- workspace layout (all offsets 256-byte aligned) ----
 struct WsLayout {
   size_t status;        // int32 status word + control counters (4 KiB block)
+  size_t ctr;           // fused-decode counters (zero between launches); size set by H, I, E only,
+                        // so the offset is the same for every T
   size_t counts;        // int32 [E]
   size_t offsets;       // int32 [E+1]
   size_t perm;          // int32 [T*k]
@@ -60,8 +75,17 @@ enum CtlWord {
   kCtlWords = 1024
 };
 
+// Tensor maps over a packed bank (slots x N x K, layout MW4T v2) whose box is one 128 x 128 tile:
+// codes as (32-bit word of a 512-byte chunk, K group, row group over all slots) with box
+// (128, 1, 16); scales as (row in the chunk, K group, row group over all slots) with box
+// (8, 1, 16). The tile of row block rb, K group g in slot s is at (0, g, s * N/8 + 16 * rb) and
+// lands in shared memory as 16 chunks of 512 bytes (codes) or 128 scales in row order.
+int make_chunk_code_map(void* map, const void* base, int N, int K, int slots);
+int make_chunk_scale_map(void* map, const void* base, int N, int K, int slots);
+
 size_t permute_scratch_count(int T, int k, int E);
 size_t decode_scratch_bytes(int T, int H, int I, int E, int k);
+size_t decode_counter_bytes(int H, int I, int E);
 
 // ---- launch helpers (defined in the .cu files) ----
 int launch_quantize_pack(const uint16_t* w, int E, int N, int K, uint8_t* packed, uint16_t* scales,
@@ -81,7 +105,6 @@ struct FfnArgs {
   bool accumulate;
   const uint16_t* logits; // fused decode: route in-kernel when non-null
   int32_t* idx_out; float* wts_out;
-  bool tc_decode;         // fused decode on the tcgen05 kernel instead of the warp-MMA one
 };
 int ffn_simple(const FfnArgs& a, cudaStream_t s);
 int ffn_sequential(const FfnArgs& a, cudaStream_t s);

@@ -13,6 +13,7 @@
 #pragma once
 
 #include <algorithm>
+#include <cuda.h>
 
 #include "common.cuh"
 #include "tc.cuh"
@@ -50,6 +51,13 @@ struct DecParams {
   int nstages;
   uint32_t mul16;               // 65536, passed at run time so that x * mul16 stays an IMAD
   unsigned long long* trace;    // optional per-CTA diagnostics (64 x u64 per CTA), null normally
+  long long wait_cycles;        // single-token kernel: limit of its bounded waits (0 = default)
+  int extra_arrivals;           // single-token kernel: arrivals expected beyond the grid (test hook)
+};
+
+// Tensor maps of the two packed banks, one 128 x 128 tile per box (make_chunk_code_map).
+struct alignas(64) DecMaps {
+  CUtensorMap c13, s13, c2, s2;
 };
 
 // trace slots per CTA: 0 start, 1 plan done, 3 weights all issued, 4 all h ready, 5 compute
@@ -427,16 +435,29 @@ __device__ __forceinline__ void encode_group(const float (&v)[4], uint8_t* hi, u
 }
 
 // ---- host side
-struct DecScratch { size_t hcnt, fcnt, hdone, p1, p2, hbuf, total; };
+// Counters (zero between launches), in their own workspace region whose offset does not depend
+// on T: hcnt [E][I/128], fcnt [H/128], hdone [4] (m <= E selected experts at any batch size).
+struct DecCounters { size_t hcnt, fcnt, hdone, total; };
+inline DecCounters dec_counters(int H, int I, int E) {
+  DecCounters C{};
+  const size_t nI = I / kRowBlock, nH = H / kRowBlock;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 256); return at; };
+  C.hcnt = take(sizeof(int) * (size_t)E * nI);
+  C.fcnt = take(sizeof(int) * nH);
+  C.hdone = take(sizeof(int) * 4);
+  C.total = off;
+  return C;
+}
+
+// Partials and operands (no initial value needed).
+struct DecScratch { size_t p1, p2, hbuf, total; };
 // hbuf_per_tile: bytes of h operand per (selected expert, K group of I)
 inline DecScratch dec_scratch(int T, int H, int I, int E, int k, size_t hbuf_per_tile) {
   DecScratch D{};
   const size_t m = (size_t)std::min(E, T * k), nI = I / kRowBlock, nH = H / kRowBlock;
   size_t off = 0;
   auto take = [&](size_t bytes) { const size_t at = off; off = align_up(off + bytes, 256); return at; };
-  D.hcnt = take(sizeof(int) * m * nI);
-  D.fcnt = take(sizeof(int) * nH);
-  D.hdone = take(sizeof(int) * 4);
   D.p1 = take(sizeof(float) * (m * 2 * nI + kMaxGrid) * T * kRowBlock);
   D.p2 = take(sizeof(float) * (nH + kMaxGrid) * T * kRowBlock);
   D.hbuf = take(m * nI * hbuf_per_tile);
@@ -456,7 +477,7 @@ extern unsigned long long* g_trace;
 
 // Single-token decode kernel (defined in ffn_decode_rows.cu)
 bool rows_supported(int T, int H, int I, int E, int k);
-size_t rows_hbuf_bytes(int H, int I, int E, int k);
+size_t rows_hbuf_per_tile();
 int launch_decode_rows(const DecParams& P, int grid, cudaStream_t s);
 
 // Warp-MMA decode kernel for T <= kMmaMaxT (defined in ffn_decode_mma.cu)

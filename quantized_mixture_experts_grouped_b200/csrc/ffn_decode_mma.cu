@@ -73,9 +73,11 @@ struct TileAcc {
 template <int NB>
 __device__ __forceinline__ void tile_issue(const uint8_t* tb, const uint16_t* sc, const uint8_t* bcol, int cs,
                                            const uint8_t* rec, int r0, int kh, int g, int c, int T, TileAcc<NB>& A) {
+  // the tile is 16 chunks of 512 bytes, one per 8-row group (rows r0 and r0 + 8: adjacent chunks)
   const int q = 2 * kh + (c >> 1);
-  const uint2 w0 = *reinterpret_cast<const uint2*>(tb + q * 2048 + r0 * 16 + (c & 1) * 8);
-  const uint2 w1 = *reinterpret_cast<const uint2*>(tb + q * 2048 + (r0 + 8) * 16 + (c & 1) * 8);
+  const uint8_t* p0 = tb + (r0 >> 3) * kChunkBytes + piece_offset(q, r0 & 7) + (c & 1) * 8;
+  const uint2 w0 = *reinterpret_cast<const uint2*>(p0);
+  const uint2 w1 = *reinterpret_cast<const uint2*>(p0 + kChunkBytes);
   const uint32_t M = 0x0F0F0F0Fu;
   const uint32_t a0 = w0.x & M, a1 = w1.x & M, a2 = (w0.x >> 4) & M, a3 = (w1.x >> 4) & M;
   const uint32_t b0 = w0.y & M, b1 = w1.y & M, b2 = (w0.y >> 4) & M, b3 = (w1.y >> 4) & M;
@@ -174,14 +176,17 @@ __device__ __forceinline__ void sum_partials2(const float* P0, int ba, int a0, i
 }
 
 template <int TT>
-__global__ void __launch_bounds__(kMThreads, 1) moe_decode_mma_kernel(const __grid_constant__ DecParams P) {
+__global__ void __launch_bounds__(kMThreads, 1) moe_decode_mma_kernel(const __grid_constant__ DecParams P,
+                                                                      const __grid_constant__ DecMaps M) {
   using C = Cfg<TT>;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   MSmem<TT>& s = *reinterpret_cast<MSmem<TT>*>(smem_raw);
   const int xcs = P.H + kColPad;                                  // activation column stride (bytes)
   uint8_t* xq = smem_raw + sizeof(MSmem<TT>);
   uint8_t* xrec = xq + (size_t)C::kCols * xcs;                    // [H/128][4 NB] group records
-  uint8_t* ring = xrec + (size_t)(P.H / kGroup) * 4 * C::NB * 16;
+  // the stage ring starts on a 128-byte boundary of the shared address space (tensor copies)
+  uint8_t* ring_raw = xrec + (size_t)(P.H / kGroup) * 4 * C::NB * 16;
+  uint8_t* ring = ring_raw + (((tc::smem_u32(ring_raw) + 127u) & ~127u) - tc::smem_u32(ring_raw));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NS = P.nstages;
 
@@ -237,8 +242,7 @@ __global__ void __launch_bounds__(kMThreads, 1) moe_decode_mma_kernel(const __gr
   pl.init(s.rs.nact, P.H, P.I, G, cta);
   volatile int* abort = &s.abort;
   const int T = P.T;
-  const size_t w13_bytes = (size_t)P.I * P.H, s13_count = (size_t)2 * P.I * pl.nH;
-  const size_t w2_bytes = (size_t)P.H * P.I / 2, s2_count = (size_t)P.H * pl.nI;
+  const int rg13 = 2 * P.I / kRowGroup, rg2 = P.H / kRowGroup;   // 8-row groups per slot
   auto stage_w = [&](int st) { return ring + (size_t)st * C::kStageBytes; };
   auto stage_s = [&](int st) { return ring + (size_t)st * C::kStageBytes + kStageW; };
   auto stage_h = [&](int st) { return ring + (size_t)st * C::kStageBytes + kStageW + kStageS; };
@@ -302,12 +306,19 @@ __global__ void __launch_bounds__(kMThreads, 1) moe_decode_mma_kernel(const __gr
         int j, lt;
         pl.locate(phase, u, j, lt);
         const int sl = s.rs.sl[j];
-        const uint8_t* wsrc = phase == 1 ? P.w13 + (size_t)sl * w13_bytes : P.w2 + (size_t)sl * w2_bytes;
-        const uint16_t* ssrc = phase == 1 ? P.s13 + (size_t)sl * s13_count : P.s2 + (size_t)sl * s2_count;
         if (lane == 0) tc::mbar_arrive_expect_tx(&s.full[st], (uint32_t)(n * (kTileBytes + kRowBlock * 2)));
         __syncwarp();
-        if (lane == 0) tc::bulk_g2s(stage_w(st), wsrc + (size_t)lt * kTileBytes, (uint32_t)(n * kTileBytes), &s.full[st], pol);
-        if (lane == 1) tc::bulk_g2s(stage_s(st), ssrc + (size_t)lt * kRowBlock, (uint32_t)(n * kRowBlock * 2), &s.full[st], pol);
+        // tile i of the stage: local tile lt + i = (row block, K group) of the expert's matrix;
+        // lanes 0..3 load the codes, lanes 4..7 the scales, one tile each
+        if (lane < 2 * kTilesPerStage && (lane & 3) < n) {
+          const int i = lane & 3, nG = phase == 1 ? pl.nH : pl.nI;
+          const int t = lt + i, rb = t / nG, gq = t - rb * nG;
+          const int z = sl * (phase == 1 ? rg13 : rg2) + rb * (kRowBlock / kRowGroup);
+          if (lane < kTilesPerStage)
+            tc::tma_load_3d(stage_w(st) + i * kTileBytes, phase == 1 ? &M.c13 : &M.c2, 0, gq, z, &s.full[st], pol);
+          else
+            tc::tma_load_3d(stage_s(st) + i * kRowBlock * 2, phase == 1 ? &M.s13 : &M.s2, 0, gq, z, &s.full[st], pol);
+        }
         if (lane == 0 && it < 8) trace_clk(P, 48 + it);
         if (phase == 2) {
           // h is waited for only when a slot holding a pending stage is needed again (or at the
@@ -536,7 +547,7 @@ __global__ void __launch_bounds__(kMThreads, 1) moe_decode_mma_kernel(const __gr
 template <int TT>
 size_t smem_fixed(int H) {
   using C = Cfg<TT>;
-  return sizeof(MSmem<TT>) + (size_t)C::kCols * (H + kColPad) + (size_t)(H / kGroup) * 4 * C::NB * 16;
+  return sizeof(MSmem<TT>) + (size_t)C::kCols * (H + kColPad) + (size_t)(H / kGroup) * 4 * C::NB * 16 + 128;
 }
 
 template <int TT>
@@ -546,7 +557,7 @@ int stages_tt(int H) {
 }
 
 template <int TT>
-int launch_tt(const DecParams& P0, int grid, cudaStream_t s) {
+int launch_tt(const DecParams& P0, const DecMaps& M, int grid, cudaStream_t s) {
   DecParams P = P0;
   P.nstages = stages_tt<TT>(P.H);
   const size_t smem = smem_fixed<TT>(P.H) + (size_t)P.nstages * Cfg<TT>::kStageBytes;
@@ -567,7 +578,7 @@ int launch_tt(const DecParams& P0, int grid, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, moe_decode_mma_kernel<TT>, P);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, moe_decode_mma_kernel<TT>, P, M);
   note_launch();
   return check_cuda(e, "moe_decode_mma_kernel launch");
 }
@@ -597,12 +608,17 @@ int mma_stages(int T, int H) {
 }
 
 int launch_decode_mma(const DecParams& P, int grid, cudaStream_t s) {
+  DecMaps M;
+  if (int rc = make_chunk_code_map(&M.c13, P.w13, 2 * P.I, P.H, P.E)) return rc;
+  if (int rc = make_chunk_scale_map(&M.s13, P.s13, 2 * P.I, P.H, P.E)) return rc;
+  if (int rc = make_chunk_code_map(&M.c2, P.w2, P.H, P.I, P.E)) return rc;
+  if (int rc = make_chunk_scale_map(&M.s2, P.s2, P.H, P.I, P.E)) return rc;
   switch (tt_of(P.T)) {
-    case 1: return launch_tt<1>(P, grid, s);
-    case 2: return launch_tt<2>(P, grid, s);
-    case 4: return launch_tt<4>(P, grid, s);
-    case 8: return launch_tt<8>(P, grid, s);
-    default: return launch_tt<16>(P, grid, s);
+    case 1: return launch_tt<1>(P, M, grid, s);
+    case 2: return launch_tt<2>(P, M, grid, s);
+    case 4: return launch_tt<4>(P, M, grid, s);
+    case 8: return launch_tt<8>(P, M, grid, s);
+    default: return launch_tt<16>(P, M, grid, s);
   }
 }
 

@@ -51,8 +51,8 @@ enum { kModeGateUp = 0, kModeDown = 1 };
 
 struct __align__(1024) GStage {
   uint8_t b[2][kBBoxBytes];     // token rows, K 0..63 and 64..127 of the group (SW128)
-  uint8_t w[2][8192];           // int4 tiles of block 0 and block 1
-  uint16_t sc[2][128];          // their scales
+  uint8_t w[2][8192];           // int4 tiles of block 0 and block 1 (16 chunks of 8 rows each)
+  uint16_t sc[2][128];          // their scales, in row order
 };
 
 struct GSmem {
@@ -69,8 +69,7 @@ struct GSmem {
 };
 
 struct GParams {
-  const uint8_t* w; const uint16_t* s;     // packed bank of the matrix (per slot)
-  size_t w_stride, s_stride;                // per slot
+  int rg_slot;                              // 8-row groups per slot (N / 8) of the matrix
   int K;                                    // H for gate/up, I for down
   int G;                                    // K / 128
   int rows_half;                            // gate/up: I (up block offset); down: unused
@@ -138,9 +137,11 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, volatile i
 }
 
 // Token-row maps of one operand with boxes of 128, 64 and 32 rows: a tile of at most 64 (32)
-// tokens loads only those rows, so its stages carry fewer bytes and turn over faster.
+// tokens loads only those rows, so its stages carry fewer bytes and turn over faster. Then the
+// weight bank's tile maps (codes, scales; see make_chunk_code_map).
 struct alignas(64) BMaps {
   CUtensorMap m[3];
+  CUtensorMap wc, ws;
 };
 
 struct TileDesc {
@@ -206,6 +207,8 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
     s.abort = 0;
     tc::fence_barrier_init();
     for (int i = 0; i < 3; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.m[i]) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.wc) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.ws) : "memory");
   }
   if (warp == 1) {
     tc::tmem_alloc<kGTmemCols>(&s.tmem_base);
@@ -241,8 +244,9 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
       const int bi = d.ntok <= 32 ? 2 : (d.ntok <= 64 ? 1 : 0);   // token rows loaded: 128 >> bi
       const CUtensorMap* xmap = &xm.m[bi];
       const uint32_t bbytes = kBBoxBytes >> bi;
-      const uint8_t* wb = P.w + (size_t)d.slot * P.w_stride;
-      const uint16_t* sb = P.s + (size_t)d.slot * P.s_stride;
+      // the pair's two 128-row blocks: row-group coordinates in the bank's tile maps
+      const int z0 = d.slot * P.rg_slot + (int)d.rb0 * (kRowBlock / kRowGroup);
+      const int z1 = d.slot * P.rg_slot + (int)d.rb1 * (kRowBlock / kRowGroup);
       bool ok = true;
       for (int g = d.g0; g < d.g1; ++g, ++it) {
         const int st = it % kGStages;
@@ -252,11 +256,10 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           tc::mbar_arrive_expect_tx(&s.full[st], 2 * bbytes + 2 * 8192 + 2 * 256);
           tma_load_2d(S.b[0], xmap, g * 128, d.p0, &s.full[st]);
           tma_load_2d(S.b[1], xmap, g * 128 + 64, d.p0, &s.full[st]);
-          const size_t t0 = d.rb0 * P.G + g, t1 = d.rb1 * P.G + g;
-          tc::bulk_g2s(S.w[0], wb + t0 * kTileBytes, 8192, &s.full[st], pol_w);
-          tc::bulk_g2s(S.w[1], wb + t1 * kTileBytes, 8192, &s.full[st], pol_w);
-          tc::bulk_g2s(S.sc[0], sb + t0 * kRowBlock, 256, &s.full[st], pol_w);
-          tc::bulk_g2s(S.sc[1], sb + t1 * kRowBlock, 256, &s.full[st], pol_w);
+          tc::tma_load_3d(S.w[0], &xm.wc, 0, g, z0, &s.full[st], pol_w);
+          tc::tma_load_3d(S.w[1], &xm.wc, 0, g, z1, &s.full[st], pol_w);
+          tc::tma_load_3d(S.sc[0], &xm.ws, 0, g, z0, &s.full[st], pol_w);
+          tc::tma_load_3d(S.sc[1], &xm.ws, 0, g, z1, &s.full[st], pol_w);
           if (it < 16) gtrace(P, 48 + it);
         }
       }
@@ -350,7 +353,9 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
         const uint8_t* wsrc = s.st[st].w[blk];
         uint4 c[4];
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq) c[kq] = *reinterpret_cast<const uint4*>(wsrc + kq * 2048 + r * 16);
+        // tile in shared memory: 16 chunks of 512 bytes, one per 8-row group
+        for (int kq = 0; kq < 4; ++kq)
+          c[kq] = *reinterpret_cast<const uint4*>(wsrc + (r >> 3) * kChunkBytes + piece_offset(kq, r & 7));
         const uint32_t sbits = s.st[st].sc[blk][r];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&s.empty[st]);
@@ -673,9 +678,14 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
     if (int rc = make_rows_map(&hmap.m[i], hp, Tk, a.I, kTokTile >> i)) return rc;
   }
 
+  // the banks hold at least E slots' worth of addressable rows (slot indices are < E)
+  if (int rc = make_chunk_code_map(&xmap.wc, a.w13, 2 * a.I, a.H, a.E)) return rc;
+  if (int rc = make_chunk_scale_map(&xmap.ws, a.s13, 2 * a.I, a.H, a.E)) return rc;
+  if (int rc = make_chunk_code_map(&hmap.wc, a.w2, a.H, a.I, a.E)) return rc;
+  if (int rc = make_chunk_scale_map(&hmap.ws, a.s2, a.H, a.I, a.E)) return rc;
+
   GParams P{};
-  P.w = a.w13; P.s = a.s13;
-  P.w_stride = (size_t)2 * a.I * a.H / 2; P.s_stride = (size_t)2 * a.I * (a.H / kGroup);
+  P.rg_slot = 2 * a.I / kRowGroup;
   P.K = a.H; P.G = a.H / kGroup; P.rows_half = a.I; P.mode = kModeGateUp;
   P.ksplit = 1; P.part_stride = 0;
   P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
@@ -683,8 +693,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   P.trace = nullptr;
   if (int rc = launch_gemm(P, xmap, max_chunks * IB, s)) return rc;
 
-  P.w = a.w2; P.s = a.s2;
-  P.w_stride = (size_t)a.H * a.I / 2; P.s_stride = (size_t)a.H * (a.I / kGroup);
+  P.rg_slot = a.H / kRowGroup;
   P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
   P.ksplit = ksplit; P.part_stride = ksplit == 2 ? (size_t)Tk * a.H : 0;   // the partials fill the fp32-sized yp
   P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;

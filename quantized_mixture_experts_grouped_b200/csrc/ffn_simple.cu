@@ -86,22 +86,23 @@ __global__ void __launch_bounds__(128) gateup_simple_kernel(
   const int r = threadIdx.x, ib = blockIdx.y;
   const int G = H / kGroup;
   const size_t wstride = (size_t)2 * I * H / 2, sstride = (size_t)2 * I * G;
-  const uint8_t* wg = w13 + ti.slot * wstride + (size_t)ib * G * kTileBytes + r * 16;
-  const uint8_t* wu = w13 + ti.slot * wstride + (size_t)(I / kRowBlock + ib) * G * kTileBytes + r * 16;
-  const uint16_t* sg = s13 + ti.slot * sstride + (size_t)ib * G * kRowBlock + r;
-  const uint16_t* su = s13 + ti.slot * sstride + (size_t)(I / kRowBlock + ib) * G * kRowBlock + r;
+  const int ng = ib * kRowBlock + r, nu = I + ng;   // gate and up rows of this thread
+  const uint8_t* wg = w13 + ti.slot * wstride + chunk_offset(ng / kRowGroup, 0, G) + (ng % kRowGroup) * 16;
+  const uint8_t* wu = w13 + ti.slot * wstride + chunk_offset(nu / kRowGroup, 0, G) + (nu % kRowGroup) * 16;
+  const uint16_t* sg = s13 + ti.slot * sstride + chunk_scale_index(ng / kRowGroup, 0, G) + ng % kRowGroup;
+  const uint16_t* su = s13 + ti.slot * sstride + chunk_scale_index(nu / kRowGroup, 0, G) + nu % kRowGroup;
   float ag[kPairsPerTile] = {}, au[kPairsPerTile] = {};
   for (int g = 0; g < G; ++g) {
     __syncthreads();
     for (int pp = 0; pp < kPairsPerTile; ++pp)
       xs[pp][r] = pp < ti.np ? bf16_bits_to_float(xp[(size_t)(ti.p0 + pp) * H + g * kGroup + r]) : 0.f;
     __syncthreads();
-    const float scg = bf16_bits_to_float(sg[(size_t)g * kRowBlock]);
-    const float scu = bf16_bits_to_float(su[(size_t)g * kRowBlock]);
+    const float scg = bf16_bits_to_float(sg[(size_t)g * kRowGroup]);
+    const float scu = bf16_bits_to_float(su[(size_t)g * kRowGroup]);
     for (int kq = 0; kq < 4; ++kq) {
       float fg[32], fu[32];
-      dequant32(*reinterpret_cast<const uint4*>(wg + (size_t)g * kTileBytes + kq * 2048), scg, fg);
-      dequant32(*reinterpret_cast<const uint4*>(wu + (size_t)g * kTileBytes + kq * 2048), scu, fu);
+      dequant32(*reinterpret_cast<const uint4*>(wg + (size_t)g * kChunkBytes + kq * 128), scg, fg);
+      dequant32(*reinterpret_cast<const uint4*>(wu + (size_t)g * kChunkBytes + kq * 128), scu, fu);
 #pragma unroll
       for (int c = 0; c < 32; ++c)
 #pragma unroll
@@ -129,18 +130,19 @@ __global__ void __launch_bounds__(128) down_simple_kernel(
   const int r = threadIdx.x, nb = blockIdx.y;
   const int G = I / kGroup;
   const size_t wstride = (size_t)H * I / 2, sstride = (size_t)H * G;
-  const uint8_t* wd = w2 + ti.slot * wstride + (size_t)nb * G * kTileBytes + r * 16;
-  const uint16_t* sd = s2 + ti.slot * sstride + (size_t)nb * G * kRowBlock + r;
+  const int n0 = nb * kRowBlock + r;
+  const uint8_t* wd = w2 + ti.slot * wstride + chunk_offset(n0 / kRowGroup, 0, G) + (n0 % kRowGroup) * 16;
+  const uint16_t* sd = s2 + ti.slot * sstride + chunk_scale_index(n0 / kRowGroup, 0, G) + n0 % kRowGroup;
   float acc[kPairsPerTile] = {};
   for (int g = 0; g < G; ++g) {
     __syncthreads();
     for (int pp = 0; pp < kPairsPerTile; ++pp)
       hs[pp][r] = pp < ti.np ? bf16_bits_to_float(hp[(size_t)(ti.p0 + pp) * I + g * kGroup + r]) : 0.f;
     __syncthreads();
-    const float sc = bf16_bits_to_float(sd[(size_t)g * kRowBlock]);
+    const float sc = bf16_bits_to_float(sd[(size_t)g * kRowGroup]);
     for (int kq = 0; kq < 4; ++kq) {
       float f[32];
-      dequant32(*reinterpret_cast<const uint4*>(wd + (size_t)g * kTileBytes + kq * 2048), sc, f);
+      dequant32(*reinterpret_cast<const uint4*>(wd + (size_t)g * kChunkBytes + kq * 128), sc, f);
 #pragma unroll
       for (int c = 0; c < 32; ++c)
 #pragma unroll

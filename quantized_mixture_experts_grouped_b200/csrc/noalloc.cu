@@ -10,9 +10,10 @@
 // point runs with that device current; that first call should therefore come before any stream
 // capture on the device. Every call on a device shares the one array, so calls that may run at
 // the same time (different streams, or different host threads) race and must be serialised by
-// the caller. Each call clears, on its stream, the words that must start at zero: the status and
-// control block at the head of the workspace and the fused-decode counters. Nothing here
-// allocates: no cudaMalloc / cudaFree, no allocating library.
+// the caller. Each call clears, on its stream, the words that must start at zero: the control
+// block at the head of the workspace (all but the status word) and the fused-decode counters.
+// The status word keeps the first device-side failure until moe_noalloc_status reads it. Nothing
+// here allocates: no cudaMalloc / cudaFree, no allocating library.
 #include <mutex>
 
 #include "common.cuh"
@@ -47,8 +48,6 @@ int scratch_for_current_device(void** out) {
 
 }  // namespace
 
-size_t decode_counters_bytes(int T, int H, int I, int E, int k);
-
 }  // namespace moe
 
 using namespace moe;
@@ -72,16 +71,22 @@ MOE_API int moe_w4a16_layer_noalloc(const uint16_t* x_bf16, const uint16_t* logi
   void* ws = nullptr;
   if (int rc = scratch_for_current_device(&ws)) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // words that must start at zero: status/control block and the fused-decode counters
+  // words that must start at zero: the control block after the status word, and the
+  // fused-decode counters, which sit together at the head of the workspace
   char* base = static_cast<char*>(ws);
-  if (int rc = check_cuda(cudaMemsetAsync(base + L.status, 0, L.counts - L.status, s),
-                          "moe_w4a16_layer_noalloc: clearing the control block"))
+  const size_t keep = sizeof(int32_t) * 2;   // status word and its wait site
+  if (int rc = check_cuda(cudaMemsetAsync(base + L.status + keep, 0, L.counts - L.status - keep, s),
+                          "moe_w4a16_layer_noalloc: clearing the control block and counters"))
     return rc;
-  const size_t ctr = decode_counters_bytes(T, H, I, E, k);
-  if (ctr > 0)
-    if (int rc = check_cuda(cudaMemsetAsync(base + L.dec, 0, ctr, s),
-                            "moe_w4a16_layer_noalloc: clearing the decode counters"))
-      return rc;
   return moe_w4a16_layer(x_bf16, logits_bf16, T, H, I, E, k, w13, s13, w2, s2, slot_of_expert, idx, wts, ws,
                          kNoAllocScratchBytes, out_bf16, flags, stream);
+}
+
+// Status of the calls above on the current device: reads (synchronously, on `stream`) and clears
+// the status word of the static array, as moe_workspace_status does for a caller workspace.
+MOE_API int moe_noalloc_status(moe_stream_t stream, int* status) {
+  if (!status) return fail(MOE_ERR_ARG, "moe_noalloc_status: null pointer");
+  void* ws = nullptr;
+  if (int rc = scratch_for_current_device(&ws)) return rc;
+  return moe_workspace_status(ws, stream, status);
 }

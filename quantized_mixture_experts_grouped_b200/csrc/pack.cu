@@ -1,8 +1,9 @@
 // Symmetric group-128 int4 quantiser + packer ("Every Expert Counts: ExactMoE for
 // Memory-Efficient W4A16 Inference", Abstract: group-128 four-bit weights for the routed
-// experts only). One CTA quantises one 128-row x 128-K tile: it stages the bf16 tile in shared
+// experts only). One CTA quantises 128 rows x one 128-K group: it stages the bf16 values in shared
 // memory with coalesced 32-bit loads, then each thread owns one row: absmax, scale, codes, and
-// four 16-byte chunks written in the "MW4T v1" layout (coalesced across the CTA).
+// four 16-byte pieces written in the "MW4T v2" layout (row r lands in the 512-byte chunk of its
+// 8-row group and K group; eight consecutive rows fill 128 contiguous bytes per quarter).
 #include "common.cuh"
 
 namespace moe {
@@ -39,8 +40,8 @@ __global__ void __launch_bounds__(128) quantize_pack_kernel(const uint16_t* __re
   const __nv_bfloat16 sb = __float2bfloat16_rn(s32);
   const float sf = __bfloat162float(sb);
 
-  const size_t tile_idx = (size_t)rb * G + g;
-  uint8_t* dst = packed + (size_t)e * ((size_t)N * K / 2) + tile_idx * kTileBytes + (size_t)r * 16;
+  const size_t chunk = ((size_t)rb * (kRowBlock / kRowGroup) + r / kRowGroup) * G + g;
+  uint8_t* dst = packed + (size_t)e * ((size_t)N * K / 2) + chunk * kChunkBytes + (size_t)(r % kRowGroup) * 16;
   for (int kq = 0; kq < 4; ++kq) {
     uint32_t words[4];
     for (int wi = 0; wi < 4; ++wi) {
@@ -55,9 +56,9 @@ __global__ void __launch_bounds__(128) quantize_pack_kernel(const uint16_t* __re
       }
       words[wi] = word;
     }
-    *reinterpret_cast<uint4*>(dst + kq * 2048) = make_uint4(words[0], words[1], words[2], words[3]);
+    *reinterpret_cast<uint4*>(dst + kq * 128) = make_uint4(words[0], words[1], words[2], words[3]);
   }
-  scales[(size_t)e * ((size_t)N * G) + tile_idx * kRowBlock + r] = __bfloat16_as_ushort(sb);
+  scales[(size_t)e * ((size_t)N * G) + chunk * kRowGroup + r % kRowGroup] = __bfloat16_as_ushort(sb);
 }
 
 }  // namespace

@@ -233,10 +233,12 @@ MOE_API int moe_slot_cache_layer(moe_slot_cache* c, const uint16_t* x, const uin
       return rc;
     if (int rc = check_cuda(cudaStreamWaitEvent(s, c->loaded, 0), "moe_slot_cache_layer: wait refill")) return rc;
     const bool last = !any();
+    // wave 0 stores its sum into the fp32 accumulator without reading it (no zero precondition
+    // on the accumulator, even after an earlier call ended early); later waves add to it; the
+    // last wave writes out
     const int flags = (path & MOE_PATH_MASK) | (wave > 0 ? MOE_FLAG_ACCUMULATE : 0);
     if (int rc = moe_w4a16_ffn(x, T, c->H, c->I, E, k, idx, wts, c->pool_w13, c->pool_s13, c->pool_w2, c->pool_s2,
-                               table_d, workspace, workspace_bytes, last ? out : nullptr,
-                               last ? flags : (flags | MOE_FLAG_ACCUMULATE), stream))
+                               table_d, workspace, workspace_bytes, last ? out : nullptr, flags, stream))
       return rc;
     if (int rc = check_cuda(cudaEventRecord(c->compute_done, s), "moe_slot_cache_layer: record")) return rc;
     ++wave;

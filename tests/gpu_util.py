@@ -64,6 +64,11 @@ class Layer:
                               self.wl.H, self.wl.I, tokens=tokens, active=active)
 
 
+# (case, max-abs error, relative L2 error) of every FFN comparison in this process, printed at
+# the end of the run (tests/conftest.py) so that each case's margin against the tolerance shows.
+FFN_RESULTS: list = []
+
+
 def assert_ffn_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
     got = got.astype(np.float64)
     ref = ref.astype(np.float64)
@@ -71,5 +76,6 @@ def assert_ffn_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
     max_abs = float(np.max(np.abs(got - ref))) if got.size else 0.0
     denom = float(np.linalg.norm(ref)) or 1.0
     rel = float(np.linalg.norm(got - ref)) / denom
+    FFN_RESULTS.append((what, max_abs, rel))
     assert max_abs <= FFN_MAX_ABS and rel <= FFN_REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
     return max_abs, rel

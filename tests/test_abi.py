@@ -84,11 +84,11 @@ def test_binding_constants_match_the_header():
     values = {n: int(v, 0) for n, v in re.findall(r"\b(MOE_[A-Z0-9_]+)\s*=\s*(0x[0-9a-fA-F]+|\d+)", text)}
     for name in ("MOE_OK", "MOE_ERR_ARG", "MOE_ERR_SHAPE", "MOE_ERR_CUDA", "MOE_ERR_TIMEOUT",
                  "MOE_PATH_AUTO", "MOE_PATH_SIMPLE", "MOE_PATH_DECODE", "MOE_PATH_GROUPED",
-                 "MOE_PATH_SEQUENTIAL", "MOE_PATH_DECODE_TC", "MOE_FLAG_ACCUMULATE"):
+                 "MOE_PATH_SEQUENTIAL", "MOE_FLAG_ACCUMULATE"):
         assert values[name] == getattr(q, name), name
     assert sorted(q.PATHS.values()) == sorted(values[n] for n in values if n.startswith("MOE_PATH_")
                                               and n != "MOE_PATH_MASK")
-    assert q.lib.moe_packed_layout_version() == 1
+    assert q.lib.moe_packed_layout_version() == 2
 
 
 def test_header_is_plain_c_and_links(tmp_path):
@@ -105,7 +105,7 @@ def test_header_is_plain_c_and_links(tmp_path):
 #include "moe_w4a16.h"
 int main(void) {
   size_t ws = 0;
-  if (moe_abi_version() != 1 || moe_packed_layout_version() != 1) return 1;
+  if (moe_abi_version() != 1 || moe_packed_layout_version() != 2) return 1;
   if (moe_packed_bytes(2048, 2048) != (size_t)2048 * 2048 / 2) return 2;
   if (moe_scales_count(2048, 1024) != (size_t)2048 * 8) return 3;
   if (moe_workspace_bytes(1, 2048, 1024, 64, 8, &ws) != MOE_OK || ws == 0) return 4;

@@ -22,25 +22,24 @@ def test_expert_bytes_match_the_packed_layout():
 
 
 def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
-    import hashlib
-    # a summary written for copies of the profiled sources is read back while they are unchanged
+    import json
+    # a record written for copies of the profiled sources is read back while they are unchanged
     copies = []
     for i, f in enumerate(bench.PROFILE_SOURCES):
         dst = tmp_path / f"src{i}"
         shutil.copyfile(os.path.join(ROOT, f), dst)
         copies.append(str(dst))
-    digest = hashlib.sha256(b"".join(open(c, "rb").read() for c in copies)).hexdigest()[:16]
-    summary = tmp_path / "summary.md"
-    summary.write_text(f"kernel source hash (two files): {digest}\ntraffic_bytes_per_launch: 12345\n")
     monkeypatch.setattr(bench, "PROFILE_SOURCES", copies)
-    monkeypatch.setattr(bench, "PROFILE", str(summary))
+    record = tmp_path / "record.json"
+    record.write_text(json.dumps({"source_hash": bench.source_hash(), "traffic_bytes_per_launch": 12345}))
+    monkeypatch.setattr(bench, "PROFILE", str(record))
     assert bench.profiled_traffic() == 12345
     # any change to a profiled source drops the figure
     with open(copies[0], "a") as fh:
         fh.write("\n// edited\n")
     assert bench.profiled_traffic() is None
-    # so does a missing summary
-    monkeypatch.setattr(bench, "PROFILE", str(tmp_path / "missing.md"))
+    # so does a missing record
+    monkeypatch.setattr(bench, "PROFILE", str(tmp_path / "missing.json"))
     assert bench.profiled_traffic() is None
 
 

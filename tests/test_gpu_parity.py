@@ -18,17 +18,17 @@ pytestmark = pytest.mark.gpu
 
 q = pytest.importorskip("quantized_mixture_experts_grouped_b200")
 
-FFN_PATHS = ["simple", "decode", "decode_tc", "grouped", "sequential"]
+FFN_PATHS = ["simple", "decode", "grouped", "sequential"]
 
 
 def _supported(path, T, k):
     """The fused decode path takes small batches only (T <= 16 and T*k <= 256)."""
-    if path in ("decode", "decode_tc") and not (1 <= T <= 16 and T * k <= 256):
+    if path == "decode" and not (1 <= T <= 16 and T * k <= 256):
         pytest.skip("fused decode path is for small batches")
 
 
 def _supported_h(path, H):
-    if path in ("decode", "decode_tc") and H > 3072:
+    if path == "decode" and H > 3072:
         pytest.skip("fused decode path stages the activations in shared memory: H <= 3072")
     if path == "grouped" and H % 256:
         pytest.skip("grouped GEMM pairs 128-row blocks of W2: H must be a multiple of 256")
@@ -219,7 +219,7 @@ def test_ffn_edge_cases_small_batch(path):
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
 
 
-@pytest.mark.parametrize("path", ["auto", "decode", "decode_tc", "simple", "grouped", "sequential"])
+@pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped", "sequential"])
 @pytest.mark.parametrize("T", [1, 5, 16, 300])
 def test_layer_call_routes_and_runs(path, T):
     """moe_w4a16_layer: routing (in-kernel on the fused path) + FFN in one call."""
@@ -253,28 +253,46 @@ def test_ffn_olmoe_decode_and_batched(path):
         assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"{name} {path}")
 
 
+_FULL = {}
+
+
+def _full_layer(name):
+    """The full-size layer and the oracle's output for every one of its tokens, computed once per
+    process (tens of seconds of oracle on the host cores) and shared by the paths."""
+    if name not in _FULL:
+        layer = Layer(mi.WORKLOADS[name])
+        _FULL[name] = (layer, layer.oracle_out())
+    return _FULL[name]
+
+
 @pytest.mark.parametrize("path", FFN_PATHS)
-def test_ffn_prefill_full_size_sampled(path):
+def test_ffn_prefill_full_size(path):
+    """All 2048 tokens of the OLMoE prefill layer (Zipf routing: experts with one to fifteen
+    128-token chunks, ragged tails, experts with few tokens) against the oracle."""
+    _supported(path, 2048, 8)
     wl = mi.WORKLOADS["olmoe_prefill"]
-    layer = Layer(wl)
+    layer, ref = _full_layer("olmoe_prefill")
     counts = np.bincount(layer.idx.ravel(), minlength=wl.E)
     assert counts.max() > 1000 and counts.min() < 200      # Zipf skew reached the kernels
+    assert np.any(counts % 128 != 0) and np.any(counts > 128)
     out, _ = _run_ffn(layer, path)
     got = bf16_dev_to_f32(out)
-    assert np.all(np.isfinite(got))
-    tokens = [0, 1, 777, 1024, 2047]
-    assert_ffn_close(got[tokens], layer.oracle_out(tokens=tokens), f"prefill {path}")
+    assert_ffn_close(got, ref, f"full: prefill T=2048 {path}")
+    # every token on its own as well: a local error cannot hide in the global norm
+    for t in range(0, wl.T, 97):
+        assert_ffn_close(got[t:t + 1], ref[t:t + 1], f"prefill token {t} {path}")
 
 
 @pytest.mark.parametrize("path", FFN_PATHS)
-def test_ffn_large_expert_full_size_sampled(path):
-    wl = mi.WORKLOADS["large_expert"]
-    layer = Layer(wl)
+def test_ffn_large_expert_full_size(path):
+    """All 512 tokens of the large-expert layer (H=4096, I=14336, top-2 of 8)."""
+    _supported(path, 512, 2)
+    layer, ref = _full_layer("large_expert")
     out, _ = _run_ffn(layer, path)
     got = bf16_dev_to_f32(out)
-    assert np.all(np.isfinite(got))
-    tokens = [0, 255, 511]
-    assert_ffn_close(got[tokens], layer.oracle_out(tokens=tokens), f"large {path}")
+    assert_ffn_close(got, ref, f"full: large_expert T=512 {path}")
+    for t in range(0, 512, 61):
+        assert_ffn_close(got[t:t + 1], ref[t:t + 1], f"large_expert token {t} {path}")
 
 
 @pytest.mark.parametrize("path", FFN_PATHS)
@@ -373,6 +391,73 @@ def test_slot_cache_layer_matches_oracle(path):
         assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"cache step {step}")
         total_waves += n_waves
     assert total_waves > 12          # some steps needed more than one wave (k*T > S)
+
+
+@pytest.mark.parametrize("path", ["auto", "grouped"])
+def test_slot_cache_olmoe_slots_full_size(path):
+    """The batched-decode slot-cache workload at its own shapes: E=64 experts, 16 slots, 16 tokens
+    per step, Zipf(1.1) routing (about 40 distinct experts per step, so three waves), H=2048,
+    I=1024, three consecutive steps of one layer. Waves, loads, LRU state and slot tables
+    bit-exact against the oracle's policy; every step's output against the oracle's FFN."""
+    wl = mi.WORKLOADS["olmoe_slots"]
+    S = wl.slots
+    base = Layer(wl, layer=4)
+    cache = _make_cache(wl, S, base)
+    ref_state = oracle.SlotState(wl.E, S)
+    copy_stream = torch.cuda.Stream()
+    ws = _ws(wl.T, wl.H, wl.I, wl.E, wl.k)
+    wave_tables = torch.empty(wl.E * (wl.E // S + 2), dtype=torch.int32, device="cuda")
+    seen_waves = 0
+    for step in range(3):
+        layer = Layer(wl, layer=4, step=step, experts=[])
+        layer.w13, layer.s13, layer.w2, layer.s2 = base.w13, base.s13, base.w2, base.s2
+        d = layer.to_device()
+        idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+        out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+        n_waves, n_loads = cache.layer(d["x"], d["logits"], wl.k, idx, wts, wave_tables, ws, out,
+                                       path=q.PATHS[path], copy_stream=copy_stream)
+        torch.cuda.synchronize()
+        assert q.moe_workspace_status(ws) == 0
+        np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
+        np.testing.assert_allclose(wts.cpu().numpy(), layer.wts, rtol=ROUTE_RTOL)
+        needed = np.zeros(wl.E, np.uint8)
+        needed[np.unique(layer.idx)] = 1
+        waves = loads = 0
+        while needed.any():
+            _, ld = ref_state.wave(needed)
+            waves += 1
+            loads += len(ld)
+        assert (n_waves, n_loads) == (waves, loads)
+        se, lu, clock = cache.state()
+        np.testing.assert_array_equal(se, ref_state.slot_expert)
+        np.testing.assert_array_equal(lu, ref_state.last_used)
+        assert clock == ref_state.clock[0]
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"full: olmoe_slots step {step} {path}")
+        seen_waves += n_waves
+    assert seen_waves >= 6           # the routed set exceeded the 16 slots
+
+
+def test_workspace_reused_across_sizes_and_paths():
+    """One workspace sized for the largest call serves calls of other batch sizes and paths in
+    turn (the counters that must start at zero sit at offsets that do not depend on T)."""
+    wl = mi.Workload("reuse", H=512, I=256, E=16, k=4, T=64)
+    layers = {T: Layer(wl, layer=1, step=T, T=T) for T in (1, 2, 4, 16, 64)}
+    ws = _ws(64, wl.H, wl.I, wl.E, wl.k)
+    seq = [(1, "auto"), (2, "auto"), (1, "decode"), (64, "grouped"), (16, "decode"), (4, "simple"),
+           (1, "auto"), (16, "grouped"), (2, "decode"), (64, "auto"), (1, "decode")]
+    for T, path in seq:
+        layer = layers[T]
+        d = layer.to_device()
+        idx = torch.empty((T, wl.k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((T, wl.k), dtype=torch.float32, device="cuda")
+        out = torch.empty((T, wl.H), dtype=torch.bfloat16, device="cuda")
+        q.moe_w4a16_layer(d["x"], d["logits"], wl.k, d["w13"], d["s13"], d["w2"], d["s2"], wl.H, wl.I, idx, wts,
+                          ws, out, flags=q.PATHS[path])
+        torch.cuda.synchronize()
+        assert q.moe_workspace_status(ws) == 0, (T, path)
+        np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"reused workspace T={T} {path}")
 
 
 def test_slot_table_update_refill_failure_is_reported():

@@ -114,3 +114,31 @@ def test_single_token_duplicate_routing_is_reported():
                     flags=q.MOE_PATH_DECODE)
     torch.cuda.synchronize()
     assert q.moe_workspace_status(ws) == q.MOE_ERR_ARG
+
+
+def test_single_token_wait_timeout_is_reported_and_workspace_recovers():
+    """Failure detection without a GPU fault: with a short wait limit (about 0.1 ms) and an
+    exchange that waits for one arrival more than the kernel launches, the bounded wait runs out,
+    the kernel records MOE_ERR_TIMEOUT in the workspace status word and exits. The next call on
+    the same workspace, with the hook off, runs normally and matches the oracle."""
+    wl = mi.WORKLOADS["olmoe_decode"]
+    probe = Layer(mi.Workload("p", H=128, I=128, E=wl.E, k=wl.k, T=1, routing=wl.routing, seed=wl.seed),
+                  layer=6, step=2, experts=[])
+    routed = sorted(set(probe.idx.ravel().tolist()))
+    layer = Layer(wl, layer=6, step=2, T=1, experts=routed, logits=probe.logits)
+    ws = q.alloc_workspace(1, wl.H, wl.I, wl.E, wl.k)
+    out = torch.empty((1, wl.H), dtype=torch.bfloat16, device="cuda")
+    try:
+        q.moe_debug_set_wait_limit(200_000, 1)
+        _call(layer, "decode", ws, out)
+        torch.cuda.synchronize()
+    finally:
+        q.moe_debug_set_wait_limit(0, 0)
+    assert q.moe_workspace_status(ws) == q.MOE_ERR_TIMEOUT
+    assert q.moe_workspace_status(ws) == 0          # read-and-clear
+    for rep in range(2):
+        out2 = torch.full((1, wl.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        _call(layer, "decode", ws, out2)
+        torch.cuda.synchronize()
+        assert q.moe_workspace_status(ws) == 0
+        assert_ffn_close(bf16_dev_to_f32(out2), layer.oracle_out(), f"T=1 after a timeout, rep {rep}")

@@ -60,6 +60,29 @@ def test_noalloc_matches_layer_call_twice():
             torch.cuda.synchronize()
             np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
             np.testing.assert_allclose(wts.cpu().numpy(), layer.wts, rtol=ROUTE_RTOL)
+            assert q.moe_noalloc_status() == 0
             got = bf16_dev_to_f32(out)
             assert_ffn_close(got, ref, f"{w.name} no-alloc vs layer call, rep {rep}")
             assert_ffn_close(got, oracle_out, f"{w.name} no-alloc vs oracle, rep {rep}")
+
+
+@pytest.mark.gpu
+def test_noalloc_grouped_path_and_reuse_across_sizes():
+    """Calls that the default path sends to the grouped GEMMs (64 tokens), and calls of other batch
+    sizes in between, through the one static array: each against the oracle, status clean."""
+    import torch
+    from gpu_util import Layer, assert_ffn_close, bf16_dev_to_f32
+
+    wl = mi.WORKLOADS["tiny"]
+    for T in (64, 1, 16, 64, 3):
+        layer = Layer(wl, T=T, step=T)
+        d = layer.to_device()
+        idx = torch.empty((T, wl.k), dtype=torch.int32, device="cuda")
+        wts = torch.empty((T, wl.k), dtype=torch.float32, device="cuda")
+        out = torch.full((T, wl.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        q.moe_w4a16_layer_noalloc(d["x"], d["logits"], wl.k, d["w13"], d["s13"], d["w2"], d["s2"], wl.H, wl.I,
+                                  idx, wts, out)
+        torch.cuda.synchronize()
+        assert q.moe_noalloc_status() == 0
+        np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
+        assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"no-alloc tiny T={T}")
