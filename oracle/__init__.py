@@ -56,9 +56,11 @@ def lib():
         L.orc_permute.argtypes = [P, c.c_int, c.c_int, c.c_int, P, P, P, P]
         L.orc_moe_ffn.argtypes = [P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, P, P,
                                   P, P, P, P, P, c.c_int, P, P, c.c_int]
+        L.orc_moe_ffn_bf16.argtypes = [P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, P, P,
+                                       P, P, P, c.c_int, P, P, c.c_int]
         L.orc_slot_wave.argtypes = [c.c_int, c.c_int, P, P, P, P, P, P, P, P]
         for f in ("orc_quantize", "orc_pack", "orc_unpack", "orc_dequant", "orc_route",
-                  "orc_permute", "orc_moe_ffn", "orc_slot_wave"):
+                  "orc_permute", "orc_moe_ffn", "orc_moe_ffn_bf16", "orc_slot_wave"):
             getattr(L, f).restype = c.c_int
         _lib = L
     return _lib
@@ -176,6 +178,27 @@ def moe_ffn(x_bf16, idx, wts, w13, s13, w2, s2, H: int, I: int, tokens=None, act
                            _p(np.ascontiguousarray(w2)), _p(np.ascontiguousarray(s2)),
                            _p(tok), nt, _p(act), _p(out), int(n_threads))
     _check(rc, "moe_ffn")
+    return out
+
+
+def moe_ffn_bf16(x_bf16, idx, wts, w13_bf16, w2_bf16, H: int, I: int, tokens=None, active=None,
+                 n_threads: int = 0) -> np.ndarray:
+    """Layer output (fp32) for `tokens` (default: all) from unquantised bf16 banks
+    w13 [E][2I][H], w2 [E][H][I] (uint16 bit patterns)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    wts = np.ascontiguousarray(wts, dtype=np.float32)
+    T, k = idx.shape
+    E = w13_bf16.shape[0]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
+    nt = T if tok is None else len(tok)
+    act = None if active is None else np.ascontiguousarray(active, dtype=np.uint8)
+    out = np.zeros((nt, H), np.float32)
+    rc = lib().orc_moe_ffn_bf16(_p(x), T, H, I, E, k, _p(idx), _p(wts),
+                                _p(np.ascontiguousarray(w13_bf16, dtype=np.uint16)),
+                                _p(np.ascontiguousarray(w2_bf16, dtype=np.uint16)),
+                                _p(tok), nt, _p(act), _p(out), int(n_threads))
+    _check(rc, "moe_ffn_bf16")
     return out
 
 

@@ -303,6 +303,58 @@ int orc_moe_ffn(const uint16_t* x, int T, int H, int I, int E, int k,
   return 0;
 }
 
+// The same MoE FFN layer on UNQUANTISED bf16 expert weights (the BF16 configuration the ExactMoE
+// abstract compares its W4A16 decode against): w13 [E][2I][H] (rows 0..I-1 gate, I..2I-1 up) and
+// w2 [E][H][I], row-major bf16, read exactly as fp32; everything else as orc_moe_ffn (fp64).
+int orc_moe_ffn_bf16(const uint16_t* x, int T, int H, int I, int E, int k,
+                     const int32_t* idx, const float* wts,
+                     const uint16_t* w13, const uint16_t* w2,
+                     const int32_t* tokens, int n_tokens, const uint8_t* active,
+                     float* out, int n_threads) {
+  if (!x || !idx || !wts || !w13 || !w2 || !out) return 1;
+  if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || k > E || T < 0) return 1;
+  const int nt = tokens ? n_tokens : T;
+  const size_t w13_stride = (size_t)2 * I * H, w2_stride = (size_t)H * I;
+  const int n_pairs = nt * k;
+  std::vector<double> y((size_t)n_pairs * H, 0.0);
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+  for (int pi = 0; pi < n_pairs; ++pi) {
+    const int ti = pi / k, j = pi % k;
+    const int t = tokens ? tokens[ti] : ti;
+    const int e = idx[(size_t)t * k + j];
+    if (e < 0 || e >= E) continue;
+    if (active && !active[e]) continue;
+    std::vector<double> xv(H), h(I);
+    for (int c = 0; c < H; ++c) xv[c] = bf16_to_f32(x[(size_t)t * H + c]);
+    const uint16_t* pw13 = w13 + (size_t)e * w13_stride;
+    for (int i = 0; i < I; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < H; ++c) g += (double)bf16_to_f32(pw13[(size_t)i * H + c]) * xv[c];
+      for (int c = 0; c < H; ++c) u += (double)bf16_to_f32(pw13[(size_t)(I + i) * H + c]) * xv[c];
+      h[i] = silu(g) * u;
+    }
+    const uint16_t* pw2 = w2 + (size_t)e * w2_stride;
+    double* yp = y.data() + (size_t)pi * H;
+    for (int n = 0; n < H; ++n) {
+      double acc = 0.0;
+      for (int i = 0; i < I; ++i) acc += (double)bf16_to_f32(pw2[(size_t)n * I + i]) * h[i];
+      yp[n] = acc;
+    }
+  }
+  for (int ti = 0; ti < nt; ++ti) {
+    const int t = tokens ? tokens[ti] : ti;
+    for (int n = 0; n < H; ++n) {
+      double acc = 0.0;
+      for (int j = 0; j < k; ++j) acc += (double)wts[(size_t)t * k + j] * y[((size_t)ti * k + j) * H + n];
+      out[(size_t)ti * H + n] = (float)acc;
+    }
+  }
+  return 0;
+}
+
 // One wave of the GPU slot cache (the abstract's "configurable GPU-resident slot cache"; the
 // pages give no policy, so this is the plainest reading: least-recently-used replacement).
 // State: slot_expert[S] (-1 = free), last_used[S], *clock. needed[E] (0/1) marks the experts

@@ -408,3 +408,61 @@ def test_slot_waves_invariants_random():
         # every expert resident at the start and needed this step is a hit (never reloaded)
         hits = resident_before & set(want.tolist())
         assert len(hits) <= S
+
+
+# ----------------------------------------------------------------------------- FFN on bf16 weights
+
+def test_ffn_bf16_weights_equal_w4_on_exactly_representable_weights():
+    """Weights q * 2^e (q in -8..7) are exact both as bf16 values and as packed codes with a
+    power-of-two scale: the bf16-weight FFN and the packed-weight FFN then see the same numbers
+    and sum them in the same order, so their outputs are identical."""
+    g = np.random.default_rng(11)
+    H, I, E, k, T = 256, 128, 4, 2, 5
+    wl = mi.Workload("x", H=H, I=I, E=E, k=k, T=T)
+    x = mi.activations(wl)
+    idx, wts = oracle.route(mi.router_logits(wl), k)
+    w13b = np.empty((E, 2 * I, H), np.uint16)
+    w2b = np.empty((E, H, I), np.uint16)
+    w13p, s13p, w2p, s2p = [], [], [], []
+    for e in range(E):
+        for (N, K, dst, lp, ls) in ((2 * I, H, w13b, w13p, s13p), (H, I, w2b, w2p, s2p)):
+            q = g.integers(-8, 8, (N, K)).astype(np.int8)
+            ex = g.integers(-12, -4, (N, K // 128))
+            sc = np.ldexp(1.0, ex).astype(np.float32)
+            w = q.astype(np.float32) * np.repeat(sc, 128, axis=1)
+            dst[e] = mi.to_bf16_bits(w)
+            assert np.array_equal(_f32(dst[e]), w)          # exact in bf16
+            pk, st = oracle.pack(q, _bf16(sc))
+            lp.append(pk)
+            ls.append(st)
+    a = oracle.moe_ffn(x, idx, wts, np.stack(w13p), np.stack(s13p), np.stack(w2p), np.stack(s2p), H, I)
+    b = oracle.moe_ffn_bf16(x, idx, wts, w13b, w2b, H, I)
+    assert np.array_equal(a, b)
+
+
+def test_ffn_bf16_weights_equal_dense_brute_force():
+    """Every expert on every token with numpy fp64 matmuls over the bf16 weights, masked by the
+    routed weights; a planted transposed operand is caught."""
+    wl = mi.Workload("b", H=256, I=128, E=6, k=3, T=7)
+    x = mi.activations(wl)
+    idx, wts = oracle.route(mi.router_logits(wl), wl.k)
+    w13b, w2b = mi.bank_weights(wl)
+    out = oracle.moe_ffn_bf16(x, idx, wts, w13b, w2b, wl.H, wl.I)
+    xf = _f32(x).astype(np.float64)
+    mask = np.zeros((wl.T, wl.E))
+    for t in range(wl.T):
+        for j in range(wl.k):
+            mask[t, idx[t, j]] += wts[t, j]
+    dense = np.zeros((wl.T, wl.H))
+    wrong = np.zeros((wl.T, wl.H))
+    for e in range(wl.E):
+        W13 = _f32(w13b[e]).astype(np.float64)
+        W2 = _f32(w2b[e]).astype(np.float64)
+        h = _silu(xf @ W13[:wl.I].T) * (xf @ W13[wl.I:].T)
+        dense += mask[:, e:e + 1] * (h @ W2.T)
+        wrong += mask[:, e:e + 1] * (h @ W2.reshape(wl.I, wl.H))   # W2 read transposed
+    np.testing.assert_allclose(out, dense, rtol=1e-5, atol=1e-7)
+    assert not np.allclose(out, wrong, rtol=1e-3, atol=1e-5)
+    # a token subset gives the same rows
+    sub = oracle.moe_ffn_bf16(x, idx, wts, w13b, w2b, wl.H, wl.I, tokens=[6, 0, 3])
+    np.testing.assert_array_equal(sub, out[[6, 0, 3]])
