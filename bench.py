@@ -313,7 +313,7 @@ def run_reference_tokens(args, wl: mi.Workload, world: int):
 
 
 def config_of(wl: mi.Workload, args, path: str):
-    return {"workload": wl.name, "layers": wl.layers, "hidden": wl.H, "intermediate": wl.I, "experts": wl.E,
+    return {"workload": wl.name, "weights": getattr(args, "weights", "w4a16"), "layers": wl.layers, "hidden": wl.H, "intermediate": wl.I, "experts": wl.E,
             "top_k": wl.k, "tokens_per_step": wl.T, "slots": wl.slots or wl.E, "routing": wl.routing,
             "path": path, "l2": "inputs larger than L2 (packed bank of all layers, fresh routing per step)"}
 
@@ -325,14 +325,18 @@ class DecodeBench:
 
     RING = 32   # distinct step inputs (fresh routing each); replayed cyclically
 
-    def __init__(self, wl: mi.Workload, path: str, device):
+    def __init__(self, wl: mi.Workload, path: str, device, weights: str = "w4a16"):
         import quantized_mixture_experts_grouped_b200 as q
         self.q, self.wl, self.dev = q, wl, device
         self.flags = q.PATHS[path]
+        self.bf16 = weights == "bf16"
         H, I, E, k, T, Ls = wl.H, wl.I, wl.E, wl.k, wl.T, wl.layers
         self.banks = []
         for l in range(Ls):
             w13b, w2b = mi.device_bank_weights(wl, l, device)
+            if self.bf16:        # the BF16 comparison: unquantised experts
+                self.banks.append((w13b, None, w2b, None))
+                continue
             w13, s13 = q.alloc_bank(E, 2 * I, H, device)
             w2, s2 = q.alloc_bank(E, H, I, device)
             q.moe_quantize_pack(w13b, w13, s13)
@@ -379,8 +383,12 @@ class DecodeBench:
             w13, s13, w2, s2 = self.banks[l]
             if events is not None:
                 events[2 * l].record(self.stream)
-            q.moe_w4a16_layer(x, lg, wl.k, w13, s13, w2, s2, wl.H, wl.I, self.idx[l], self.wts[l], self.ws,
-                              out[l], flags=self.flags, stream=self.stream)
+            if self.bf16:
+                q.moe_bf16_layer(x, lg, wl.k, w13, w2, wl.H, wl.I, self.idx[l], self.wts[l], self.ws, out[l],
+                                 flags=self.flags, stream=self.stream)
+            else:
+                q.moe_w4a16_layer(x, lg, wl.k, w13, s13, w2, s2, wl.H, wl.I, self.idx[l], self.wts[l], self.ws,
+                                  out[l], flags=self.flags, stream=self.stream)
             if events is not None:
                 events[2 * l + 1].record(self.stream)
 
@@ -473,7 +481,7 @@ class DecodeBench:
 
 def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
     device = torch.device("cuda", local)
-    bench = DecodeBench(wl, args.path, device)
+    bench = DecodeBench(wl, args.path, device, args.weights)
     bench.capture()
     s = bench.stream
     peaks, peaks_kind = load_peaks()
@@ -537,7 +545,7 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
     torch.cuda.empty_cache()
     # the prefill layer measured in the same process (a figure for the tensor-bound side)
     secondary = None
-    if not args.no_secondary and wl.name == "olmoe_decode":
+    if not args.no_secondary and wl.name == "olmoe_decode" and wl.T == 1 and args.weights == "w4a16":
         pw = mi.WORKLOADS["olmoe_prefill"]
         r = measure_single_layer(pw, "auto", 20, 3, world, local)
         secondary = {"workload": pw.name, "us_per_layer": r["ms"] * 1e3, "tokens_per_s": pw.T * world / (r["ms"] / 1e3),
@@ -549,7 +557,8 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
         return
     tokens = wl.T * args.steps * world
     value = tokens / (ms_total / 1e3)
-    bytes_per_layer = distinct_mean * expert_bytes(wl.H, wl.I)
+    per_expert = (2 * (3 * wl.H * wl.I)) if args.weights == "bf16" else expert_bytes(wl.H, wl.I)
+    bytes_per_layer = distinct_mean * per_expert
     # duration of the one launch of a layer: the timed step over its layers (the launches of a
     # step run back to back, so this includes the gap between two launches)
     us_layer = ms_total / args.steps / wl.layers * 1e3
@@ -565,7 +574,8 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
                      "traffic": profiled_traffic() if (wl.T == 1 and args.path in ("auto", "decode")) else None,
                      "kernel": ("moe_decode_rows_kernel" if wl.T == 1 else "moe_decode_mma_kernel")
                                + " (the one launch per layer; duration = timed step / layers)"
-                               if args.path in ("auto", "decode") else "all launches of the layer (timed step / layers)",
+                               if args.path in ("auto", "decode") and args.weights == "w4a16"
+                               else "all launches of the layer (timed step / layers)",
                      "algorithmic_bytes_per_launch": bytes_per_layer, "us_per_launch": us_layer,
                      "launches_per_layer": launches_per_layer,
                      "us_per_launch_event_pair": layer_ms * 1e3,
@@ -578,7 +588,7 @@ def run_ours(args, wl: mi.Workload, rank: int, world: int, local: int):
     }
     if secondary is not None:
         line["secondary"] = secondary
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.weights == "w4a16":
         line["cpu_baseline"] = cpu_baseline(wl)
     print(json.dumps(line), flush=True)
 
@@ -608,7 +618,8 @@ def cpu_baseline_tokens(wl: mi.Workload, budget_s: float = 12.0):
                       f"work, experts packed by the oracle)"}
 
 
-def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, world: int, local: int) -> dict:
+def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, world: int, local: int,
+                         weights: str = "w4a16") -> dict:
     """Large-batch workloads (prefill, large expert): one layer of T tokens per step through
     moe_w4a16_layer (route, permute, gather, two grouped GEMMs, combine), timed with CUDA events
     (max over ranks) with inputs resident, then end to end with host copies every step."""
@@ -616,10 +627,14 @@ def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, wo
     device = torch.device("cuda", local)
     H, I, E, k, T = wl.H, wl.I, wl.E, wl.k, wl.T
     w13b, w2b = mi.device_bank_weights(wl, 0, device)
-    w13, s13 = q.alloc_bank(E, 2 * I, H, device)
-    w2, s2 = q.alloc_bank(E, H, I, device)
-    q.moe_quantize_pack(w13b, w13, s13)
-    q.moe_quantize_pack(w2b, w2, s2)
+    bf16 = weights == "bf16"
+    if bf16:               # the BF16 comparison: unquantised experts
+        w13, s13, w2, s2 = w13b, None, w2b, None
+    else:
+        w13, s13 = q.alloc_bank(E, 2 * I, H, device)
+        w2, s2 = q.alloc_bank(E, H, I, device)
+        q.moe_quantize_pack(w13b, w13, s13)
+        q.moe_quantize_pack(w2b, w2, s2)
     del w13b, w2b
     x_host = torch.from_numpy(mi.activations(wl, 0, 0).view(np.int16)).view(torch.bfloat16).pin_memory()
     lg_host = torch.from_numpy(mi.router_logits(wl, 0, 0).view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -640,7 +655,10 @@ def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, wo
     sampler = ClockSampler(local)
 
     def call(xx, ll, oo=out):
-        q.moe_w4a16_layer(xx, ll, k, w13, s13, w2, s2, H, I, idx, wts, ws, oo, flags=flags, stream=s)
+        if bf16:
+            q.moe_bf16_layer(xx, ll, k, w13, w2, H, I, idx, wts, ws, oo, flags=flags, stream=s)
+        else:
+            q.moe_w4a16_layer(xx, ll, k, w13, s13, w2, s2, H, I, idx, wts, ws, oo, flags=flags, stream=s)
 
     h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
     in_ready = [torch.cuda.Event(), torch.cuda.Event()]
@@ -718,7 +736,7 @@ def measure_single_layer(wl: mi.Workload, path: str, steps: int, warmup: int, wo
 
 
 def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
-    r = measure_single_layer(wl, args.path, args.steps, args.warmup, world, local)
+    r = measure_single_layer(wl, args.path, args.steps, args.warmup, world, local, args.weights)
     if rank != 0:
         return
     T, ms, e2e_ms, achieved, peak = wl.T, r["ms"], r["e2e_ms"], r["achieved"], r["peak"]
@@ -739,7 +757,7 @@ def run_single_layer(args, wl: mi.Workload, rank: int, world: int, local: int):
         "clocks": r["clocks"],
         "device_status": r["status"],
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.weights == "w4a16":
         line["cpu_baseline"] = cpu_baseline_tokens(wl)
     print(json.dumps(line), flush=True)
 
@@ -864,6 +882,8 @@ def main():
     ap.add_argument("--workload", default="olmoe_decode",
                     choices=["olmoe_decode", "olmoe_slots", "olmoe_prefill", "large_expert"])
     ap.add_argument("--path", default="auto", choices=["auto", "simple", "decode", "grouped", "sequential"])
+    ap.add_argument("--weights", default="w4a16", choices=["w4a16", "bf16"],
+                    help="bf16: the same layer on unquantised experts (the BF16 comparison)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the prefill layer measured after the default decode workload")

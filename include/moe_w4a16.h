@@ -208,6 +208,29 @@ int moe_w4a16_layer_noalloc(const uint16_t* x_bf16, const uint16_t* logits_bf16,
  * finished normally on the device, else the MOE_ERR_* code of the first failure. */
 int moe_noalloc_status(moe_stream_t stream, int* status);
 
+/* ---- BF16 comparison layer (abstract: the W4A16 decode is compared with the same model in
+ * BF16). The same layer on UNQUANTISED experts, through the same grouped scheduler and tcgen05
+ * GEMMs (the weights loaded by TMA straight into the MMA operand, no dequantisation):
+ *   w13_bf16: bf16 [slots][2I][H] ([W_gate; W_up] rows, row-major), w2_bf16: bf16 [slots][H][I];
+ *   16-byte aligned. Everything else as moe_w4a16_ffn / moe_w4a16_layer (same workspace);
+ *   flags: MOE_PATH_AUTO or MOE_PATH_GROUPED, optionally | MOE_FLAG_ACCUMULATE. The per-pair down
+ * projection is rounded to bf16 before the combine, as on the W4A16 grouped path.
+ * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE (H not a multiple of 256, as on the grouped path),
+ * MOE_ERR_CUDA. */
+int moe_bf16_ffn(const uint16_t* x_bf16, int T, int H, int I, int E, int k,
+                 const int32_t* idx, const float* wts,
+                 const uint16_t* w13_bf16, const uint16_t* w2_bf16,
+                 const int32_t* slot_of_expert,
+                 void* workspace, size_t workspace_bytes,
+                 uint16_t* out_bf16, int flags, moe_stream_t stream);
+int moe_bf16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16,
+                   int T, int H, int I, int E, int k,
+                   const uint16_t* w13_bf16, const uint16_t* w2_bf16,
+                   const int32_t* slot_of_expert,
+                   int32_t* idx, float* wts,
+                   void* workspace, size_t workspace_bytes,
+                   uint16_t* out_bf16, int flags, moe_stream_t stream);
+
 /* ---- GPU slot cache (abstract: "configurable GPU-resident slot cache", experts kept in
  * pinned host memory). One cache per layer: S device slots, each holding one expert's packed
  * W13, W2 and their scales; misses are copied from the pinned host bank with

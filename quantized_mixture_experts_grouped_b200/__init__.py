@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "moe_w4a16_layer": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, Z, P, I, P], I),
         "moe_w4a16_layer_noalloc": ([P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, I, P], I),
         "moe_noalloc_status": ([P, c.POINTER(I)], I),
+        "moe_bf16_ffn": ([P, I, I, I, I, I, P, P, P, P, P, P, Z, P, I, P], I),
+        "moe_bf16_layer": ([P, P, I, I, I, I, I, P, P, P, P, P, P, Z, P, I, P], I),
         "moe_slot_cache_create": ([I, I, I, I, P, P, P, P, P, P, P, P, c.POINTER(P)], I),
         "moe_slot_cache_destroy": ([P], None),
         "moe_slot_cache_fail_copy_after": ([P, I], None),
@@ -173,6 +175,21 @@ def moe_w4a16_layer_noalloc(x, logits, k: int, w13, s13, w2, s2, H: int, I: int,
     T, E = logits.shape
     _err(lib.moe_w4a16_layer_noalloc(_p(x), _p(logits), T, H, I, E, k, _p(w13), _p(s13), _p(w2), _p(s2),
                                      _p(slot_of_expert), _p(idx), _p(wts), _p(out), flags, _s(stream)))
+
+
+def moe_bf16_ffn(x, idx, wts, w13, w2, H: int, I: int, E: int, ws, out, slot_of_expert=None,
+                 flags: int = MOE_PATH_AUTO, stream=None):
+    """The layer's FFN on unquantised bf16 experts: w13 [slots][2I][H], w2 [slots][H][I] (bf16)."""
+    T, k = idx.shape
+    _err(lib.moe_bf16_ffn(_p(x), T, H, I, E, k, _p(idx), _p(wts), _p(w13), _p(w2), _p(slot_of_expert),
+                          _p(ws), ws.numel() * ws.element_size(), _p(out), flags, _s(stream)))
+
+
+def moe_bf16_layer(x, logits, k: int, w13, w2, H: int, I: int, idx, wts, ws, out, slot_of_expert=None,
+                   flags: int = MOE_PATH_AUTO, stream=None):
+    T, E = logits.shape
+    _err(lib.moe_bf16_layer(_p(x), _p(logits), T, H, I, E, k, _p(w13), _p(w2), _p(slot_of_expert), _p(idx),
+                            _p(wts), _p(ws), ws.numel() * ws.element_size(), _p(out), flags, _s(stream)))
 
 
 def moe_noalloc_status(stream=None) -> int:

@@ -60,7 +60,9 @@ WsLayout ws_layout(int T, int H, int I, int E, int k) {
   L.yp = take(sizeof(float) * Tk * H);
   L.acc = take(sizeof(float) * (size_t)T * H);
   L.seq = take(sizeof(int32_t) * (size_t)E * E);
-  L.dec = take(decode_scratch_bytes(T, H, I, E, k));
+  // fused-decode scratch for min(T, 16) tokens: a workspace sized for T also serves every smaller
+  // batch (the total never shrinks as T grows)
+  L.dec = take(decode_scratch_bytes(std::min(T, 16), H, I, E, k));
   L.total = off;
   return L;
 }
@@ -233,4 +235,58 @@ MOE_API int moe_w4a16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16,
   }
   if (int rc = launch_route(logits_bf16, T, E, k, idx, wts, s)) return rc;
   return run_ffn(a, flags, s);
+}
+
+// ---- BF16 comparison layer: the same grouped scheduler and tcgen05 GEMMs on unquantised weights
+namespace {
+
+int check_bf16_args(const uint16_t* x, int T, int H, int I, int E, int k, const uint16_t* w13, const uint16_t* w2,
+                    void* ws, size_t ws_bytes, int flags) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return fail(MOE_ERR_ARG, "bad sizes T=%d E=%d k=%d", T, E, k);
+  if (E > kMaxExperts) return fail(MOE_ERR_SHAPE, "E=%d exceeds %d", E, kMaxExperts);
+  if (!dims_ok(H, I)) return fail(MOE_ERR_SHAPE, "H=%d and I=%d must be positive multiples of 128", H, I);
+  if (!w13 || !w2 || !ws) return fail(MOE_ERR_ARG, "null weight or workspace pointer");
+  if (T > 0 && !x) return fail(MOE_ERR_ARG, "null x");
+  const int path = flags & MOE_PATH_MASK;
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_GROUPED)
+    return fail(MOE_ERR_ARG, "the bf16-weight layer runs on the grouped path only (path %d)", path);
+  const WsLayout L = ws_layout(T, H, I, E, k);
+  if (ws_bytes < L.total)
+    return fail(MOE_ERR_ARG, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes, L.total);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0) return fail(MOE_ERR_ARG, "workspace must be 256-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w13) | reinterpret_cast<uintptr_t>(w2)) & 15)
+    return fail(MOE_ERR_ARG, "x and the weights must be 16-byte aligned");
+  return MOE_OK;
+}
+
+}  // namespace
+
+MOE_API int moe_bf16_ffn(const uint16_t* x_bf16, int T, int H, int I, int E, int k, const int32_t* idx,
+                         const float* wts, const uint16_t* w13_bf16, const uint16_t* w2_bf16,
+                         const int32_t* slot_of_expert, void* workspace, size_t workspace_bytes, uint16_t* out_bf16,
+                         int flags, moe_stream_t stream) {
+  if (int rc = check_bf16_args(x_bf16, T, H, I, E, k, w13_bf16, w2_bf16, workspace, workspace_bytes, flags)) return rc;
+  if (T > 0 && (!idx || !wts)) return fail(MOE_ERR_ARG, "moe_bf16_ffn: null idx/wts");
+  if (T == 0) return MOE_OK;
+  FfnArgs a{};
+  a.x = x_bf16; a.T = T; a.H = H; a.I = I; a.E = E; a.k = k;
+  a.idx = idx; a.wts = wts;
+  a.w13 = reinterpret_cast<const uint8_t*>(w13_bf16); a.w2 = reinterpret_cast<const uint8_t*>(w2_bf16);
+  a.slot = slot_of_expert; a.ws = static_cast<char*>(workspace); a.ws_bytes = workspace_bytes;
+  a.out = out_bf16; a.accumulate = (flags & MOE_FLAG_ACCUMULATE) != 0;
+  a.bf16_weights = true;
+  if (!ffn_grouped_supported(a)) return fail(MOE_ERR_SHAPE, "grouped GEMM path does not support these sizes");
+  return ffn_grouped(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+MOE_API int moe_bf16_layer(const uint16_t* x_bf16, const uint16_t* logits_bf16, int T, int H, int I, int E, int k,
+                           const uint16_t* w13_bf16, const uint16_t* w2_bf16, const int32_t* slot_of_expert,
+                           int32_t* idx, float* wts, void* workspace, size_t workspace_bytes, uint16_t* out_bf16,
+                           int flags, moe_stream_t stream) {
+  if (int rc = check_bf16_args(x_bf16, T, H, I, E, k, w13_bf16, w2_bf16, workspace, workspace_bytes, flags)) return rc;
+  if (T > 0 && (!logits_bf16 || !idx || !wts)) return fail(MOE_ERR_ARG, "moe_bf16_layer: null logits/idx/wts");
+  if (T == 0) return MOE_OK;
+  if (int rc = launch_route(logits_bf16, T, E, k, idx, wts, reinterpret_cast<cudaStream_t>(stream))) return rc;
+  return moe_bf16_ffn(x_bf16, T, H, I, E, k, idx, wts, w13_bf16, w2_bf16, slot_of_expert, workspace, workspace_bytes,
+                      out_bf16, flags, stream);
 }

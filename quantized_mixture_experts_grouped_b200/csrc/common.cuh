@@ -105,6 +105,7 @@ struct FfnArgs {
   bool accumulate;
   const uint16_t* logits; // fused decode: route in-kernel when non-null
   int32_t* idx_out; float* wts_out;
+  bool bf16_weights;      // w13 / w2 hold unquantised bf16 rows (grouped path only; no scales)
 };
 int ffn_simple(const FfnArgs& a, cudaStream_t s);
 int ffn_sequential(const FfnArgs& a, cudaStream_t s);

@@ -52,21 +52,24 @@ constexpr int kRHWarps = 2;                       // h warps 17, 18
 constexpr int kRWarps = 1 + kRCompute + kRHWarps;
 constexpr int kRThreads = kRWarps * 32;
 constexpr int kMaxU1 = 32;                        // phase-1 units per CTA
+constexpr int kChunkU = 2;                        // phase-1 units per copy chunk
+constexpr int kMaxChunks = kMaxU1 / kChunkU;
 constexpr int kMaxU2 = 4;                         // phase-2 units per CTA
 constexpr int kMaxSel = 32;                       // selected experts (k <= 32)
 constexpr int kRedBufs = 4;                       // phase-1 sum buffers (two per h warp)
-constexpr int kHBlock = 24;                       // encoded 8-feature h block: hi[8], lo[8], {a, a*8*sum v}
+constexpr int kHBlock = 32;                       // h block of 8 features: hi[8], lo[8], {a, a*8*sum v}, pad
 constexpr int kF = 8;                             // features per phase-1 unit
 constexpr int kORows = 16;                        // output rows per phase-2 unit
 constexpr long long kDefaultWaitCycles = 4000000000ll;   // ~2 s at the B200's peak clock
 
 struct __align__(128) RSmem {
-  uint64_t ufull[kMaxU1];                         // phase-1 unit landed
+  uint64_t cfull[kMaxChunks];                     // phase-1 chunk landed
+  uint64_t sfull;                                 // phase-1 scales landed
   uint64_t vfull[kMaxU2];                         // phase-2 unit landed
   uint64_t hfull;                                 // every h block landed
   uint64_t wready;                                // router weights in wsel
   uint64_t redfull[kRedBufs], redempty[kRedBufs];
-  float red1[kRedBufs][kRCompute][2 * kF];        // [buffer][warp][gate rows, up rows]
+  float red1[kRedBufs][kRCompute][kChunkU * 2 * kF];   // [buffer][warp][unit][gate rows, up rows]
   float red2[kRCompute][kORows];                  // [warp][row] phase-2 sums
   uint32_t key[kMaxSel];                          // winning router key of choice j
   int act[kMaxSel];                               // selected experts, ascending id
@@ -76,43 +79,25 @@ struct __align__(128) RSmem {
   int nact;
   int u1b, u1e, u2b, u2e;                         // this CTA's units
   int abort;
-  // followed in dynamic shared memory by the h blocks [m][I/8] x 24 B and the weight pieces
+  // followed in dynamic shared memory by the h blocks [m][I/8] x 32 B and the weight pieces
 };
 
-// The split of both phases over the CTAs, identical in every CTA (bytes per unit: B1, B2).
+// The split of both phases over the CTAs, identical in every CTA: the phase-1 units evenly (so that
+// phase 1, which the exchange waits for, ends at the same time everywhere), the phase-2 units one
+// or none per CTA on top.
 struct RPlan {
-  int nU1, nU2;
-  long long B1, B2;
-  __device__ __host__ static int lo2(int c, int nU2, int G) { return (int)((long long)c * nU2 / G); }
-  // phase-1 unit boundary of CTA c: the byte share c/G of the total minus the phase-2 bytes of
-  // CTAs below c, in units of B1 (rounded); non-decreasing whenever one CTA's share is at least
-  // its largest phase-2 load, else the phase-1 units are split evenly on their own
-  __device__ __host__ int lo1(int c, int G, bool joint) const {
-    if (!joint) return (int)((long long)c * nU1 / G);
-    const long long total = (long long)nU1 * B1 + (long long)nU2 * B2;
-    const long long num = (long long)c * total - (long long)G * B2 * lo2(c, nU2, G);
-    long long u = (num + (long long)G * B1 / 2) / ((long long)G * B1);
-    if (u < 0) u = 0;
-    if (u > nU1) u = nU1;
-    return (int)u;
-  }
-  __device__ __host__ bool joint(int G) const {
-    const long long total = (long long)nU1 * B1 + (long long)nU2 * B2;
-    const long long max2 = (long long)((nU2 + G - 1) / G) * B2;
-    return total >= (long long)G * max2;
-  }
+  uint32_t nU1, nU2;
   __device__ __host__ void init(int m, int H, int I) {
-    const int nH = H / kGroup, nI = I / kGroup;
-    nU1 = m * (I / kF);
+    nU1 = (uint32_t)m * (I / kF);
     nU2 = H / kORows;
-    B1 = 2LL * nH * (kChunkBytes + 16);            // gate + up row groups: codes and scales
-    B2 = (long long)m * 2 * nI * (kChunkBytes + 16);   // two row groups of every selected expert
   }
+  __device__ __host__ uint32_t lo1(int c, int G) const { return (uint32_t)c * nU1 / (uint32_t)G; }
+  __device__ __host__ uint32_t lo2(int c, int G) const { return (uint32_t)c * nU2 / (uint32_t)G; }
 };
 
 __device__ __forceinline__ void imma0(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                       uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
@@ -125,6 +110,9 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 }
 __device__ __forceinline__ void red_release_add_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Bounded wait on an mbarrier phase (every lane of the calling warp): false when the limit runs
@@ -186,8 +174,14 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
   const long long limit = P.wait_cycles > 0 ? P.wait_cycles : kDefaultWaitCycles;
   volatile int* abort = &s.abort;
 
+  // set-up that reads nothing the previous kernel writes: barriers, and L2 prefetches of the
+  // token's logits and activations (a prefetch only warms L2, which stays coherent with the
+  // previous kernel's writes; the values are read after the dependency wait)
+  unsigned long long t_entry = 0;
+  if (tid == 0 && P.trace) t_entry = tc::globaltimer();
   if (tid == 0) {
-    for (int i = 0; i < kMaxU1; ++i) tc::mbar_init(&s.ufull[i], 1);
+    for (int i = 0; i < kMaxChunks; ++i) tc::mbar_init(&s.cfull[i], 1);
+    tc::mbar_init(&s.sfull, 1);
     for (int i = 0; i < kMaxU2; ++i) tc::mbar_init(&s.vfull[i], 1);
     tc::mbar_init(&s.hfull, 1);
     tc::mbar_init(&s.wready, 1);
@@ -198,16 +192,42 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
     s.abort = 0;
     tc::fence_barrier_init();
   }
+  if (warp == 0 && P.logits && lane * 64 < P.E) prefetch_l2(P.logits + lane * 64);
+  if (warp == 1 && lane * 64 < H) prefetch_l2(P.x + lane * 64);
   __syncthreads();
+  const int G = gridDim.x, cta = blockIdx.x;
+  // every expert resident and the token's logits given: the routing selects exactly k distinct
+  // experts, so the plan (which needs only their number) is made before the dependency wait
+  const bool fast = P.logits && !P.slot && P.E <= 64;
+  const uint32_t code1 = (uint32_t)nH * kChunkBytes;                        // one row group, all of H
+  if (warp == 0 && fast) {
+    RPlan pl;
+    pl.init(P.k, H, I);
+    const uint32_t bnd = lane == 0 ? pl.lo1(cta, G) : lane == 1 ? pl.lo1(cta + 1, G)
+                         : lane == 2 ? pl.lo2(cta, G) : pl.lo2(cta + 1, G);
+    const int n1 = (int)(__shfl_sync(kFull, bnd, 1) - __shfl_sync(kFull, bnd, 0));
+    const int nch = (n1 + kChunkU - 1) / kChunkU;
+    if (lane < 4) (&s.u1b)[lane] = (int)bnd;
+    if (lane == 0) s.nact = P.k;
+    if (lane < nch)
+      tc::mbar_arrive_expect_tx(&s.cfull[lane], (uint32_t)(min(kChunkU, n1 - lane * kChunkU) * 2 * code1));
+    if (lane == 0 && n1 > 0) tc::mbar_arrive_expect_tx(&s.sfull, (uint32_t)(2 * n1 * nH * 16));
+  }
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) trace_at(P, 0);
-  const int G = gridDim.x, cta = blockIdx.x;
+  if (tid == 0 && P.trace) {   // diagnostics: entry, the previous launch's last warp, wait done
+    const unsigned long long prev_end = P.trace[blockIdx.x * 64 + 10];
+    P.trace[blockIdx.x * 64 + 11] = P.trace[blockIdx.x * 64 + 7];
+    P.trace[blockIdx.x * 64 + 10] = 0;
+    trace_at(P, 0);
+    P.trace[blockIdx.x * 64 + 8] = t_entry;
+    P.trace[blockIdx.x * 64 + 9] = prev_end;
+  }
   unsigned long long* seq = reinterpret_cast<unsigned long long*>(P.hdone + 2);
   unsigned long long seq0 = 0;
   if (tid == 0) seq0 = ld_relaxed_u64(seq);
 
-  // ---- compute warps: the token's K group(s) as B fragments (16-bit fixed point, registers)
+  // ---- compute warps: the token's K group as B fragments (16-bit fixed point, registers)
   const int cw = warp - 1, gq = lane >> 2, cq = lane & 3;
   int gk = -1;                                     // this warp's K group of every phase-1 unit
   uint32_t xb0[4] = {0, 0, 0, 0}, xb1[4] = {0, 0, 0, 0};
@@ -265,115 +285,154 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
     }
   }
 
-  // ---- warp 0: routing, plan, every weight copy
+  const size_t w13_slot = (size_t)I * H, s13_slot = (size_t)2 * I * nH;     // bytes / scales per slot
+  const size_t w2_slot = (size_t)H * I / 2, s2_slot = (size_t)H * nI;
+
+  // ---- warp 0: routing, plan, the phase-1 copies
   if (warp == 0) {
     const int k = P.k, E = P.E;
     int e = -1;
     uint32_t mykey = 0;
     float wgiven = 0.f;
-    if (P.logits) {
-      if (E <= 64) mykey = topk_keys<2>(P.logits, E, k, lane);
-      else if (E <= 128) mykey = topk_keys<4>(P.logits, E, k, lane);
-      else mykey = topk_keys<8>(P.logits, E, k, lane);
-      if (lane < k) e = 0xffff - (int)(mykey & 0xffffu);
-    } else if (lane < k) {
-      e = P.idx_in[lane];
-      wgiven = P.wts_in[lane];
+    int m = 0, below = 0, sl = -1;
+    bool in = false;
+    if (lane == 0) trace_clk(P, 16);
+    if (P.logits && !P.slot && E <= 64) {
+      // every expert resident, one token: the k winners are distinct; their presence mask and
+      // ranks follow from the winning keys directly
+      uint32_t key0 = lane < E ? route_key(P.logits[lane], lane) : 0u;
+      uint32_t key1 = lane + 32 < E ? route_key(P.logits[lane + 32], lane + 32) : 0u;
+      unsigned long long msk = 0;
+      for (int j = 0; j < k; ++j) {
+        const uint32_t win = __reduce_max_sync(kFull, max(key0, key1));
+        if (key0 == win) key0 = 0;
+        if (key1 == win) key1 = 0;
+        if (j == lane) mykey = win;
+        msk |= 1ull << (0xffff - (win & 0xffffu));
+      }
+      if (lane == 0) trace_clk(P, 17);
+      in = lane < k;
+      if (in) {
+        e = 0xffff - (int)(mykey & 0xffffu);
+        below = __popcll(msk & ((1ull << e) - 1ull));
+        sl = e;
+      }
+      m = k;
+    } else {
+      if (P.logits) {
+        if (E <= 64) mykey = topk_keys<2>(P.logits, E, k, lane);
+        else if (E <= 128) mykey = topk_keys<4>(P.logits, E, k, lane);
+        else mykey = topk_keys<8>(P.logits, E, k, lane);
+        if (lane < k) e = 0xffff - (int)(mykey & 0xffffu);
+        if (lane == 0) trace_clk(P, 17);
+      } else if (lane < k) {
+        e = P.idx_in[lane];
+        wgiven = P.wts_in[lane];
+      }
+      if (lane < k && (unsigned)e < (unsigned)E) sl = slot_of(P.slot, e);
+      in = sl >= 0;
+      const int n_in = __popc(__ballot_sync(kFull, in));
+      const int nw = (E + 31) >> 5;
+      uint32_t mw = 0;   // lane wd < nw: presence word wd
+      for (int wd = 0; wd < nw; ++wd) {
+        const uint32_t v = __reduce_or_sync(kFull, (in && (e >> 5) == wd) ? 1u << (e & 31) : 0u);
+        if (lane == wd) mw = v;
+      }
+      for (int wd = 0; wd < nw; ++wd) {
+        const uint32_t v = __shfl_sync(kFull, mw, wd);
+        if (in && wd < (e >> 5)) below += __popc(v);
+        if (in && wd == (e >> 5)) below += __popc(v & ((1u << (e & 31)) - 1u));
+      }
+      const int total = (int)__reduce_add_sync(kFull, (uint32_t)__popc(mw));
+      const bool dup = total != n_in;
+      m = dup ? 0 : total;
+      if (dup) in = false;
+      if (lane == 0 && dup) report_status(P.ctl, MOE_ERR_ARG, kSiteOver);
     }
-    int sl = -1;
-    if (lane < k && (unsigned)e < (unsigned)E) sl = slot_of(P.slot, e);
-    const bool in = sl >= 0;
-    const int n_in = __popc(__ballot_sync(kFull, in));
-    const int nw = (E + 31) >> 5;
-    uint32_t mw = 0;   // lane wd < nw: presence word wd
-    for (int wd = 0; wd < nw; ++wd) {
-      const uint32_t v = __reduce_or_sync(kFull, (in && (e >> 5) == wd) ? 1u << (e & 31) : 0u);
-      if (lane == wd) mw = v;
-    }
-    int below = 0;
-    for (int wd = 0; wd < nw; ++wd) {
-      const uint32_t v = __shfl_sync(kFull, mw, wd);
-      if (in && wd < (e >> 5)) below += __popc(v);
-      if (in && wd == (e >> 5)) below += __popc(v & ((1u << (e & 31)) - 1u));
-    }
-    const int total = (int)__reduce_add_sync(kFull, (uint32_t)__popc(mw));
-    const bool dup = total != n_in;
-    const int m = dup ? 0 : total;
-    if (in && !dup) {
+    if (in) {
       s.act[below] = e;
       s.sl[below] = sl;
     }
-    if (lane < kMaxSel) {
-      s.rank[lane] = (in && !dup) ? below : -1;
-      s.key[lane] = mykey;
-      s.wsel[lane] = wgiven;
-    }
-    if (lane == 0 && dup) report_status(P.ctl, MOE_ERR_ARG, kSiteOver);
-    RPlan pl;
-    pl.init(m, H, I);
-    const bool joint = pl.joint(G);
-    const int u1b = pl.lo1(cta, G, joint), u1e = pl.lo1(cta + 1, G, joint);
-    const int u2b = RPlan::lo2(cta, pl.nU2, G), u2e = m > 0 ? RPlan::lo2(cta + 1, pl.nU2, G) : u2b;
-    if (lane == 0) {
-      s.nact = m;
-      s.u1b = u1b; s.u1e = u1e; s.u2b = u2b; s.u2e = u2e;
-      trace_at(P, 1);
-    }
-    __syncwarp();
-    // every copy of this CTA, issued by the 32 lanes side by side: phase-1 unit i is copies
-    // 4i .. 4i + 3 (gate codes, up codes, gate scales, up scales), then phase-2 unit v and expert j
-    // is two copies (codes and scales of the unit's two row groups)
-    const int n1 = u1e - u1b, n2 = u2e - u2b;
-    const uint64_t pol = tc::policy_evict_first();
-    if (lane == 0) {
-      for (int i = 0; i < n1; ++i) tc::mbar_arrive_expect_tx(&s.ufull[i], (uint32_t)pl.B1);
-      for (int v = 0; v < n2; ++v) tc::mbar_arrive_expect_tx(&s.vfull[v], (uint32_t)pl.B2);
-    }
-    __syncwarp();
-    const size_t w13_slot = (size_t)I * H, s13_slot = (size_t)2 * I * nH;     // bytes / scales per slot
-    const size_t w2_slot = (size_t)H * I / 2, s2_slot = (size_t)H * nI;
-    const int nc = 4 * n1 + 2 * n2 * m;
-    for (int c = lane; c < nc; c += 32) {
-      if (c < 4 * n1) {
-        const int i = c >> 2, part = c & 3, u = u1b + i, j = u / nFB, fb = u - j * nFB;
-        const int R = (part & 1) ? (I / kRowGroup + fb) : fb;       // gate or up row group
-        const int slot = s.sl[j];
-        uint8_t* dst = pieces + (size_t)i * pl.B1;
-        if (part < 2) {
-          tc::bulk_g2s(dst + (size_t)part * nH * kChunkBytes, P.w13 + slot * w13_slot + chunk_offset(R, 0, nH),
-                       (uint32_t)(nH * kChunkBytes), &s.ufull[i], pol);
-        } else {
-          tc::bulk_g2s(dst + (size_t)2 * nH * kChunkBytes + (size_t)(part & 1) * nH * 16,
-                       P.s13 + slot * s13_slot + chunk_scale_index(R, 0, nH), (uint32_t)(nH * 16), &s.ufull[i], pol);
-        }
-      } else {
-        const int c2 = c - 4 * n1, vj = c2 >> 1, v = vj / m, j = vj - v * m, R = 2 * (u2b + v);
-        const int slot = s.sl[j];
-        uint8_t* dst = pieces + (size_t)n1 * pl.B1 + (size_t)v * pl.B2 + (size_t)j * 2 * nI * (kChunkBytes + 16);
-        if ((c2 & 1) == 0)
-          tc::bulk_g2s(dst, P.w2 + slot * w2_slot + chunk_offset(R, 0, nI), (uint32_t)(2 * nI * kChunkBytes),
-                       &s.vfull[v], pol);
-        else
-          tc::bulk_g2s(dst + (size_t)2 * nI * kChunkBytes, P.s2 + slot * s2_slot + chunk_scale_index(R, 0, nI),
-                       (uint32_t)(2 * nI * 16), &s.vfull[v], pol);
+    s.rank[lane] = in ? below : -1;
+    s.key[lane] = mykey;
+    s.wsel[lane] = wgiven;
+    if (lane == 0) trace_clk(P, 18);
+    int u1b, u1e, u2b, u2e;
+    if (fast) {
+      u1b = s.u1b; u1e = s.u1e; u2b = s.u2b; u2e = s.u2e;
+    } else {
+      RPlan pl;
+      pl.init(m, H, I);
+      // the four unit boundaries of this CTA, one per lane
+      const uint32_t bnd = lane == 0 ? pl.lo1(cta, G) : lane == 1 ? pl.lo1(cta + 1, G)
+                           : lane == 2 ? pl.lo2(cta, G) : pl.lo2(cta + 1, G);
+      u1b = (int)__shfl_sync(kFull, bnd, 0); u1e = (int)__shfl_sync(kFull, bnd, 1);
+      u2b = (int)__shfl_sync(kFull, bnd, 2); u2e = m > 0 ? (int)__shfl_sync(kFull, bnd, 3) : u2b;
+      if (lane == 0) {
+        s.nact = m;
+        s.u1b = u1b; s.u1e = u1e; s.u2b = u2b; s.u2e = u2e;
       }
     }
-    if (lane == 0) trace_at(P, 2);
+    if (lane == 0) trace_clk(P, 19);
+    __syncwarp();
+    // phase-1 copies: chunk c (units 2c, 2c + 1 of this CTA) is one copy of its gate row groups
+    // and one of its up row groups (two each when its units belong to two experts); the scales of
+    // each expert's run of units are one copy for the gate rows and one for the up rows
+    const int n1 = u1e - u1b, nch = (n1 + kChunkU - 1) / kChunkU;
+    const int j0 = n1 > 0 ? u1b / nFB : 0, nruns = n1 > 0 ? (u1e - 1) / nFB - j0 + 1 : 0;
+    const uint64_t pol = tc::policy_evict_first();
+    uint8_t* sc1 = pieces + (size_t)n1 * 2 * code1;                          // phase-1 scales
+    if (!fast && lane == 0 && n1 > 0) tc::mbar_arrive_expect_tx(&s.sfull, (uint32_t)(2 * n1 * nH * 16));
+    __syncwarp();
+    for (int c = lane; c < nch + 2 * nruns; c += 32) {
+      if (c < nch) {
+        const int i0 = c * kChunkU, nk = min(kChunkU, n1 - i0);
+        uint8_t* dst = pieces + (size_t)i0 * 2 * code1;
+        if (!fast) tc::mbar_arrive_expect_tx(&s.cfull[c], (uint32_t)(nk * 2 * code1));
+        const int ua = u1b + i0, ub = ua + nk - 1, ja = ua / nFB, jb = ub / nFB;
+        if (ja == jb) {   // both units of one expert: their row groups follow each other
+          const int fb = ua - ja * nFB;
+          const uint8_t* src = P.w13 + s.sl[ja] * w13_slot;
+          tc::bulk_g2s(dst, src + chunk_offset(fb, 0, nH), nk * code1, &s.cfull[c], pol);
+          tc::bulk_g2s(dst + (size_t)nk * code1, src + chunk_offset(I / kRowGroup + fb, 0, nH), nk * code1,
+                       &s.cfull[c], pol);
+        } else {
+          for (int q = 0; q < nk; ++q) {
+            const int u = ua + q, j = u / nFB, fb = u - j * nFB;
+            const uint8_t* src = P.w13 + s.sl[j] * w13_slot;
+            tc::bulk_g2s(dst + (size_t)q * code1, src + chunk_offset(fb, 0, nH), code1, &s.cfull[c], pol);
+            tc::bulk_g2s(dst + (size_t)(nk + q) * code1, src + chunk_offset(I / kRowGroup + fb, 0, nH), code1,
+                         &s.cfull[c], pol);
+          }
+        }
+      } else {
+        const int r = (c - nch) >> 1, up = (c - nch) & 1, j = j0 + r;
+        const int ua = max(u1b, j * nFB), ue = min(u1e, (j + 1) * nFB), fb = ua - j * nFB;
+        const int R = up ? I / kRowGroup + fb : fb;
+        tc::bulk_g2s(sc1 + ((size_t)up * n1 + (ua - u1b)) * nH * 16,
+                     P.s13 + s.sl[j] * s13_slot + chunk_scale_index(R, 0, nH), (uint32_t)((ue - ua) * nH * 16),
+                     &s.sfull, pol);
+      }
+    }
+    if (lane == 0) trace_clk(P, 21);
   }
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int m = s.nact, u1b = s.u1b, u1e = s.u1e, u2b = s.u2b, u2e = s.u2e;
-  const int n1 = u1e - u1b, n2 = u2e - u2b;
-  RPlan pl;
-  pl.init(m, H, I);
+  const int n1 = u1e - u1b, n2 = u2e - u2b, nch = (n1 + kChunkU - 1) / kChunkU;
+  const uint8_t* sc1 = pieces + (size_t)n1 * 2 * code1;
+  uint8_t* p2 = pieces + ((((size_t)n1 * 2 * code1 + (size_t)2 * n1 * nH * 16) + 127) & ~(size_t)127);
+  const uint32_t code2 = (uint32_t)(2 * nI * kChunkBytes);                 // one expert's two row groups
+  uint16_t* sc2 = reinterpret_cast<uint16_t*>(p2 + (size_t)n2 * m * code2);   // phase-2 scales
   const uint32_t hbytes = (uint32_t)(m * nFB * kHBlock);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ router weights, exchange
+    // ------------------------------------------------------------ router weights, phase-2 copies,
+    // exchange
     const int k = P.k;
     if (P.logits) {
       // renormalised weight of choice j = exp(l_j - l_max) / sum over the k chosen
-      const uint32_t mykey = lane < kMaxSel ? s.key[lane] : 0u;
+      const uint32_t mykey = s.key[lane];
       const float mx = key_logit(__shfl_sync(kFull, mykey, 0));
       const float el = lane < k ? expf(key_logit(mykey) - mx) : 0.f;
       float sum = el;
@@ -389,7 +448,7 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
         }
       }
     } else {
-      const float w = lane < kMaxSel ? s.wsel[lane] : 0.f;   // the given weights, choice order
+      const float w = s.wsel[lane];   // the given weights, choice order
       __syncwarp();
       if (lane < k) {
         const int r = s.rank[lane];
@@ -398,9 +457,22 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
     }
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(&s.wready);
+    // the phase-2 weights go out once the first phase-1 chunk has landed, so that the HBM queue
+    // serves phase 1 first and the exchange overlaps the phase-2 stream
     bool ok = true;
     if (n2 > 0) {
-      if (lane == 0) {
+      if (nch > 0) ok = rwait(&s.cfull[0], 0, abort, limit);
+      const uint64_t pol = tc::policy_evict_first();
+      if (lane == 0)
+        for (int v = 0; v < n2; ++v) tc::mbar_arrive_expect_tx(&s.vfull[v], (uint32_t)(m * code2));
+      __syncwarp();
+      for (int c = lane; c < n2 * m; c += 32) {
+        const int v = c / m, j = c - v * m;
+        tc::bulk_g2s(p2 + (size_t)c * code2, P.w2 + s.sl[j] * w2_slot + chunk_offset(2 * (u2b + v), 0, nI), code2,
+                     &s.vfull[v], pol);
+      }
+      if (lane == 0) trace_clk(P, 22);
+      if (lane == 0 && ok) {
         const unsigned long long target =
             seq0 - seq0 % (unsigned long long)G + (unsigned long long)G + (unsigned long long)P.extra_arrivals;
         const long long t0 = clock64();
@@ -412,7 +484,7 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
           // acquire (pairs with the CTAs' release adds), then order the async-proxy copy after it
           asm volatile("fence.acq_rel.gpu;" ::: "memory");
           fence_proxy_async_global();
-          trace_at(P, 4);
+          trace_clk(P, 28);
           tc::mbar_arrive_expect_tx(&s.hfull, hbytes);
           tc::bulk_g2s(hsm, P.hbuf, hbytes, &s.hfull, tc::policy_evict_first());
         } else {
@@ -424,7 +496,8 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
     }
     if (lane == 0) {   // no copy may still be landing in shared memory when the CTA leaves
       volatile int never = 0;
-      for (int i = 0; i < n1; ++i) tc::mbar_wait(&s.ufull[i], 0, &never);
+      for (int c = 0; c < nch; ++c) tc::mbar_wait(&s.cfull[c], 0, &never);
+      if (n1 > 0) tc::mbar_wait(&s.sfull, 0, &never);
       for (int v = 0; v < n2; ++v) tc::mbar_wait(&s.vfull[v], 0, &never);
       if (n2 > 0 && ok) tc::mbar_wait(&s.hfull, 0, &never);
     }
@@ -432,78 +505,118 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
   } else if (warp <= kRCompute) {
     // ------------------------------------------------------------ compute warps 1..16
     const uint32_t M = 0x0F0F0F0Fu;
+    const int ct = tid - 32;                      // 0..511
+    // the phase-2 scales of this CTA's units: plain loads into shared memory, long before use
+    // ([unit][expert][row group 0 then 1][K group][8 rows], two bf16 per 32-bit word)
+    for (int w = ct; w < n2 * m * nI * 8; w += kRCompute * 32) {
+      const int per = nI * 8, vj = w / per, rem = w - vj * per, v = vj / m, j = vj - v * m;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(P.s2 + s.sl[j] * s2_slot +
+                                                              chunk_scale_index(2 * (u2b + v), 0, nI));
+      reinterpret_cast<uint32_t*>(sc2)[w] = src[rem];
+    }
     bool ok = true;
-    // phase 1: unit i, K group gk: rows 0..7 of the MMA = gate rows, 8..15 = up rows
-    for (int i = 0; i < n1; ++i) {
-      const int b = i % kRedBufs;
-      if (i >= kRedBufs && !rwait(&s.redempty[b], ((i / kRedBufs) - 1) & 1, abort, limit)) { ok = false; break; }
-      if (!rwait(&s.ufull[i], 0, abort, limit)) { ok = false; break; }
+    // phase 1, one chunk (up to two units) per step; unit q, K group gk: rows 0..7 of the MMA =
+    // gate rows, 8..15 = up rows. The MMAs of a step are independent (one accumulator per K
+    // quarter and unit), summed afterwards, so the warp's MMAs overlap instead of forming a chain.
+    if (n1 > 0) ok = rwait(&s.sfull, 0, abort, limit);
+    for (int c = 0; c < nch && ok; ++c) {
+      const int b = c % kRedBufs, nk = min(kChunkU, n1 - c * kChunkU);
+      if (c >= kRedBufs && !rwait(&s.redempty[b], ((c / kRedBufs) - 1) & 1, abort, limit)) { ok = false; break; }
+      if (!rwait(&s.cfull[c], 0, abort, limit)) { ok = false; break; }
+      if (cw == 0 && lane == 0 && c < 16) trace_clk(P, 32 + c);
       if (gk >= 0) {
-        const uint8_t* unit = pieces + (size_t)i * pl.B1;
-        const uint8_t* gch = unit + (size_t)gk * kChunkBytes + gq * 16 + 4 * cq;
-        const uint8_t* uch = gch + (size_t)nH * kChunkBytes;
-        int d[4] = {0, 0, 0, 0};
+        const uint8_t* chunk = pieces + (size_t)c * kChunkU * 2 * code1 + (size_t)gk * kChunkBytes + gq * 16 + 4 * cq;
+        int d[kChunkU][4][4];
 #pragma unroll
-        for (int kq = 0; kq < 4; ++kq) {
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(gch + kq * 128);
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(uch + kq * 128);
-          imma(d, wa & M, wb & M, (wa >> 4) & M, (wb >> 4) & M, xb0[kq], xb1[kq]);
+        for (int q = 0; q < kChunkU; ++q) {
+          if (q < nk) {
+            const uint8_t* gch = chunk + (size_t)q * code1;
+            const uint8_t* uch = chunk + (size_t)(nk + q) * code1;
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+              const uint32_t wa = *reinterpret_cast<const uint32_t*>(gch + kq * 128);
+              const uint32_t wb = *reinterpret_cast<const uint32_t*>(uch + kq * 128);
+              imma0(d[q][kq], wa & M, wb & M, (wa >> 4) & M, (wb >> 4) & M, xb0[kq], xb1[kq]);
+            }
+          }
         }
         if (cq == 0) {   // columns 0 / 1 = hi / lo of the token
-          const uint16_t* scl = reinterpret_cast<const uint16_t*>(unit + (size_t)2 * nH * kChunkBytes);
-          const float sg = bf16_bits_to_float(scl[gk * kRowGroup + gq]);
-          const float su = bf16_bits_to_float(scl[nH * kRowGroup + gk * kRowGroup + gq]);
-          s.red1[b][cw][gq] = sg * xa * (float)(d[0] * 256 + d[1] - xcorr);
-          s.red1[b][cw][kF + gq] = su * xa * (float)(d[2] * 256 + d[3] - xcorr);
+#pragma unroll
+          for (int q = 0; q < kChunkU; ++q) {
+            if (q < nk) {
+              const int i = c * kChunkU + q;
+              const int dg0 = d[q][0][0] + d[q][1][0] + d[q][2][0] + d[q][3][0];
+              const int dg1 = d[q][0][1] + d[q][1][1] + d[q][2][1] + d[q][3][1];
+              const int du0 = d[q][0][2] + d[q][1][2] + d[q][2][2] + d[q][3][2];
+              const int du1 = d[q][0][3] + d[q][1][3] + d[q][2][3] + d[q][3][3];
+              const uint16_t* sg = reinterpret_cast<const uint16_t*>(sc1 + (size_t)i * nH * 16);
+              const uint16_t* su = reinterpret_cast<const uint16_t*>(sc1 + (size_t)(n1 + i) * nH * 16);
+              s.red1[b][cw][q * 2 * kF + gq] = bf16_bits_to_float(sg[gk * kRowGroup + gq]) * xa * (float)(dg0 * 256 + dg1 - xcorr);
+              s.red1[b][cw][q * 2 * kF + kF + gq] = bf16_bits_to_float(su[gk * kRowGroup + gq]) * xa * (float)(du0 * 256 + du1 - xcorr);
+            }
+          }
         }
-      } else if (lane < 2 * kF) {
+      } else if (lane < kChunkU * 2 * kF) {
         s.red1[b][cw][lane] = 0.f;
       }
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.redfull[b]);
     }
-    if (cw == 0 && lane == 0) trace_at(P, 3);
-    // phase 2: unit v = 16 output rows over every selected expert. Warp cw takes the (expert,
-    // K group) pairs [cw P / 16, (cw + 1) P / 16), P = m nI. Lane (g, c): A rows g (first row
-    // group) and g + 8 (second); B column g holds, in K quarter c, the hi (g even) or lo (g odd)
-    // bytes of the 8-feature h block c of the k-step, so D[r][2c], D[r][2c + 1] are block c's
-    // hi and lo sums and the lane applies block c's scale.
-    // (every compute warp runs every phase-2 unit and meets both named barriers, also after a
-    // failed wait: its MMAs and stores are then skipped)
+    if (cw == 0 && lane == 0) trace_clk(P, 27);
+    // phase 2: unit v = 16 output rows over every selected expert;
+    // warp cw takes the (expert, K group) pairs [cw P / 16, (cw + 1) P / 16), P = m nI. Lane (g, c):
+    // A rows g (first row group) and g + 8 (second); B column g holds, in K quarter c, the hi
+    // (g even) or lo (g odd) bytes of h block c of the k-step, so D[r][2c], D[r][2c + 1] are block
+    // c's hi and lo sums and the lane applies block c's scale. (Every compute warp runs every unit
+    // and meets the named barriers, also after a failed wait; its work is then skipped.)
     bool h_in = false;
     for (int v = 0; v < n2; ++v) {
       ok = ok && rwait(&s.vfull[v], 0, abort, limit);
-      if (ok && !h_in) {
-        ok = rwait(&s.hfull, 0, abort, limit);
-        h_in = ok;
-        if (ok && cw == 0 && lane == 0) trace_at(P, 5);
+      if (cw == 0 && lane == 0 && v == 0) trace_clk(P, 12);
+      if (!h_in) {
+        ok = ok && rwait(&s.hfull, 0, abort, limit);
+        if (ok && cw == 0 && lane == 0) trace_clk(P, 29);
+        h_in = true;
+        tc::named_bar_sync(1, kRCompute * 32);   // every warp's phase-2 scales are in shared memory
+        if (cw == 0 && lane == 0) trace_clk(P, 13);
       }
-      const uint8_t* unit = pieces + (size_t)n1 * pl.B1 + (size_t)v * pl.B2;
-      const int np = m * nI, p0 = cw * np / kRCompute, p1 = ok ? (cw + 1) * np / kRCompute : p0;
+      const uint8_t* unit = p2 + (size_t)v * m * code2;
+      const uint16_t* scu = sc2 + (size_t)v * m * 2 * nI * kRowGroup;
+      const int np = m * nI, q0 = cw * np / kRCompute, q1 = ok ? (cw + 1) * np / kRCompute : q0;
       float y0 = 0.f, y1 = 0.f;
-      for (int p = p0; p < p1; ++p) {
-        const int j = p / nI, g2 = p - j * nI;
-        const uint8_t* ex = unit + (size_t)j * 2 * nI * (kChunkBytes + 16);
-        const uint8_t* ch0 = ex + (size_t)g2 * kChunkBytes + gq * 16 + 4 * cq;
+      int j = q0 / nI, g2 = q0 - j * nI;
+#pragma unroll 2
+      for (int p = q0; p < q1; ++p) {
+        const uint8_t* ch0 = unit + (size_t)j * code2 + (size_t)g2 * kChunkBytes + gq * 16 + 4 * cq;
         const uint8_t* ch1 = ch0 + (size_t)nI * kChunkBytes;
-        const uint16_t* scl = reinterpret_cast<const uint16_t*>(ex + (size_t)2 * nI * kChunkBytes);
+        const uint16_t* scl = scu + (size_t)j * 2 * nI * kRowGroup;
         const uint8_t* hb = hsm + ((size_t)j * nFB + g2 * 16) * kHBlock;   // the group's 16 h blocks
+        uint32_t wa[4], wb[4];
+        uint2 hv[4];
+        float2 rec[4];
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          wa[kq] = *reinterpret_cast<const uint32_t*>(ch0 + kq * 128);
+          wb[kq] = *reinterpret_cast<const uint32_t*>(ch1 + kq * 128);
+          const uint8_t* blk = hb + (kq * 4 + cq) * kHBlock;
+          hv[kq] = (gq >> 1) == cq ? *reinterpret_cast<const uint2*>(blk + (gq & 1) * 8) : make_uint2(0u, 0u);
+          rec[kq] = *reinterpret_cast<const float2*>(blk + 16);   // {a, a * 8 sum v}
+        }
+        const float s0 = bf16_bits_to_float(scl[g2 * kRowGroup + gq]);
+        const float s1 = bf16_bits_to_float(scl[nI * kRowGroup + g2 * kRowGroup + gq]);
+        int d[4][4];
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq)
+          imma0(d[kq], wa[kq] & M, wb[kq] & M, (wa[kq] >> 4) & M, (wb[kq] >> 4) & M, hv[kq].x, hv[kq].y);
         float t0 = 0.f, t1 = 0.f;
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
-          const uint32_t wa = *reinterpret_cast<const uint32_t*>(ch0 + kq * 128);
-          const uint32_t wb = *reinterpret_cast<const uint32_t*>(ch1 + kq * 128);
-          const uint8_t* blk = hb + (kq * 4 + cq) * kHBlock;
-          uint2 hv = make_uint2(0u, 0u);
-          if ((gq >> 1) == cq) hv = *reinterpret_cast<const uint2*>(blk + (gq & 1) * 8);
-          int d[4];
-          imma0(d, wa & M, wb & M, (wa >> 4) & M, (wb >> 4) & M, hv.x, hv.y);
-          const float2 rec = *reinterpret_cast<const float2*>(blk + 16);   // {a, a * 8 sum v}
-          t0 += fmaf(rec.x, (float)(d[0] * 256 + d[1]), -rec.y);
-          t1 += fmaf(rec.x, (float)(d[2] * 256 + d[3]), -rec.y);
+          t0 += fmaf(rec[kq].x, (float)(d[kq][0] * 256 + d[kq][1]), -rec[kq].y);
+          t1 += fmaf(rec[kq].x, (float)(d[kq][2] * 256 + d[kq][3]), -rec[kq].y);
         }
-        y0 = fmaf(bf16_bits_to_float(scl[g2 * kRowGroup + gq]), t0, y0);
-        y1 = fmaf(bf16_bits_to_float(scl[nI * kRowGroup + g2 * kRowGroup + gq]), t1, y1);
+        y0 = fmaf(s0, t0, y0);
+        y1 = fmaf(s1, t1, y1);
+        if (++g2 == nI) { g2 = 0; ++j; }
       }
       // the four lanes of a row hold four different h blocks: sum them (fixed order)
       y0 += __shfl_xor_sync(kFull, y0, 1);
@@ -514,6 +627,7 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
         s.red2[cw][gq] = y0;
         s.red2[cw][gq + 8] = y1;
       }
+      if (cw == 0 && lane == 0 && v == 0) trace_clk(P, 14);
       tc::named_bar_sync(1, kRCompute * 32);
       if (cw == 0 && lane < kORows && !*abort) {
         float y = 0.f;
@@ -521,65 +635,67 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
         for (int w = 0; w < kRCompute; ++w) y += s.red2[w][lane];
         store_output(P, 0, (u2b + v) * kORows + lane, y);
       }
+      if (cw == 0 && lane == 0 && v == 0) trace_clk(P, 15);
       tc::named_bar_sync(1, kRCompute * 32);
     }
     if (!ok && lane == 0) report_status(P.ctl, MOE_ERR_TIMEOUT, kSiteStage);
   } else {
     // ------------------------------------------------------------ h warps 17, 18
-    // unit i goes to h warp i % 2: the 16 warps' sums (fixed order), h = w * silu(gate) * up of
-    // its 8 features, encoded as one 24-byte block; then one arrival per CTA
+    // chunk c goes to h warp c % 2: the 16 warps' sums (fixed order), h = w * silu(gate) * up of
+    // its units' 8 features, encoded as the down projection's B operand; then one arrival per CTA
     const int hw = warp - 1 - kRCompute;
     bool ok = rwait(&s.wready, 0, abort, limit);
-    for (int i = hw; i < n1 && ok; i += kRHWarps) {
-      const int b = i % kRedBufs;
-      if (!rwait(&s.redfull[b], (i / kRedBufs) & 1, abort, limit)) { ok = false; break; }
+    for (int c = hw; c < nch && ok; c += kRHWarps) {
+      const int b = c % kRedBufs;
+      if (!rwait(&s.redfull[b], (c / kRedBufs) & 1, abort, limit)) { ok = false; break; }
+      // lane l: entry l of the chunk (unit l / 16, gate (l % 16 < 8) or up row l % 8)
       float sum = 0.f;
-      if (lane < 2 * kF)
 #pragma unroll
-        for (int w = 0; w < kRCompute; ++w) sum += s.red1[b][w][lane];
+      for (int w = 0; w < kRCompute; ++w) sum += s.red1[b][w][lane];
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(&s.redempty[b]);
-      const float up = __shfl_sync(kFull, sum, (lane & 7) + kF);
-      const int u = u1b + i, j = u / nFB, fb = u - j * nFB;
-      const float wt = s.wsel[j];
+      const float up = __shfl_sync(kFull, sum, (lane & ~15) | ((lane & 7) + kF));
+      // lanes 0..7 and 16..23: h of the chunk's units 0 and 1, encoded per 8-feature block as
+      // v = rint(h / a), a = max|h| / 32639, hi and lo bytes in the MMA's element order (byte
+      // stores into the block), then {a, a * 8 sum v}
+      const int q = lane >> 4, i = c * kChunkU + q;
+      const bool mine = (lane & 15) < kF && i < n1;
+      const int u = u1b + (mine ? i : 0), j = u / nFB, fb = u - j * nFB;
       float hv = 0.f;
-      if (lane < kF && wt != 0.f) hv = __fdividef(sum * up, 1.f + __expf(-sum)) * wt;
+      if (mine) {
+        const float wt = s.wsel[j];
+        hv = (wt != 0.f) ? __fdividef(sum * up, 1.f + __expf(-sum)) * wt : 0.f;
+      }
       float mx = fabsf(hv);
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
       const float inv = mx > 0.f ? 32639.f / mx : 0.f;
-      const int iv = lane < kF ? max(-32639, min(32639, __float2int_rn(hv * inv))) : 0;
-      const int h8 = (iv + 128) >> 8, l8 = iv - 256 * h8;
+      const int iv = mine ? max(-32639, min(32639, __float2int_rn(hv * inv))) : 0;
       int sv = iv;
       sv += __shfl_xor_sync(kFull, sv, 1);
       sv += __shfl_xor_sync(kFull, sv, 2);
       sv += __shfl_xor_sync(kFull, sv, 4);
-      // the hi and lo bytes in the permuted element order, gathered into two 64-bit words
-      const int pos = rperm(lane & 7);
-      unsigned long long hw64 = lane < kF ? (unsigned long long)(h8 & 0xff) << (8 * pos) : 0ull;
-      unsigned long long lw64 = lane < kF ? (unsigned long long)(l8 & 0xff) << (8 * pos) : 0ull;
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        hw64 |= __shfl_xor_sync(kFull, hw64, o);
-        lw64 |= __shfl_xor_sync(kFull, lw64, o);
+      if (mine) {
+        uint8_t* blk = P.hbuf + ((size_t)j * nFB + fb) * kHBlock;
+        const int h8 = (iv + 128) >> 8, l8 = iv - 256 * h8, pos = rperm(lane & 7);
+        blk[pos] = (uint8_t)h8;
+        blk[8 + pos] = (uint8_t)l8;
+        if ((lane & 7) == 0) {
+          const float a = mx * (1.f / 32639.f);
+          *reinterpret_cast<float2*>(blk + 16) = make_float2(a, a * (float)(8 * sv));
+        }
       }
-      if (lane == 0) {
-        const float a = mx * (1.f / 32639.f);
-        unsigned long long* dst = reinterpret_cast<unsigned long long*>(P.hbuf + ((size_t)j * nFB + fb) * kHBlock);
-        const float2 rec = make_float2(a, a * (float)(8 * sv));
-        dst[0] = hw64;
-        dst[1] = lw64;
-        dst[2] = *reinterpret_cast<const unsigned long long*>(&rec);
-      }
+      if (lane == 0 && c < 16) trace_clk(P, 48 + c);
     }
     // both h warps meet, then one release: every block of this CTA is ordered before it. Every
     // CTA arrives whenever an expert is selected (also after a failed wait, which the status word
     // records), so the counter stays a multiple of G between launches.
+    if (lane == 0 && hw == 0) trace_clk(P, 25);
     tc::named_bar_sync(2, kRHWarps * 32);
     if (hw == 0 && lane == 0 && m > 0) {
       red_release_add_u64(seq, 1ull);
-      trace_at(P, 6);
+      trace_clk(P, 30);
     }
     if (!ok && lane == 0) report_status(P.ctl, MOE_ERR_TIMEOUT, kSiteH);
   }
@@ -595,33 +711,36 @@ __global__ void __launch_bounds__(kRThreads, 1) moe_decode_rows_kernel(const __g
       }
     }
   }
-  if (tid == 0) trace_at(P, 7);
+  if (tid == 0) { trace_clk(P, 31); trace_at(P, 7); }
+  if (lane == 0 && P.trace) atomicMax(P.trace + blockIdx.x * 64 + 10, tc::globaltimer());   // last warp out
 }
 
 // ---------------------------------------------------------------- host side
 size_t rows_static_smem() { return sizeof(RSmem); }
 size_t rows_h_bytes(int I, int m_max) { return ((size_t)m_max * (I / kF) * kHBlock + 127) & ~(size_t)127; }
 
-// Largest piece area and unit counts any CTA needs for m selected experts.
+// Shared memory of a CTA's pieces: phase-1 codes and scales, then (128-aligned) phase-2 codes and
+// scales.
+size_t rows_pieces_bytes(int H, int I, int m, int n1, int n2) {
+  const size_t nH = H / kGroup, nI = I / kGroup;
+  const size_t p1 = (size_t)n1 * 2 * nH * kChunkBytes + (size_t)2 * n1 * nH * 16;
+  return ((p1 + 127) & ~(size_t)127) + (size_t)n2 * m * 2 * nI * (kChunkBytes + 16);
+}
+
+// Whether every CTA's share for m selected experts fits the piece area and the unit limits.
 bool rows_plan_fits(int H, int I, int m, int G, size_t cap) {
   RPlan pl;
   pl.init(m, H, I);
-  const bool joint = pl.joint(G);
   for (int c = 0; c < G; ++c) {
-    const int n1 = pl.lo1(c + 1, G, joint) - pl.lo1(c, G, joint);
-    const int n2 = RPlan::lo2(c + 1, pl.nU2, G) - RPlan::lo2(c, pl.nU2, G);
+    const int n1 = (int)pl.lo1(c + 1, G) - (int)pl.lo1(c, G);
+    const int n2 = (int)pl.lo2(c + 1, G) - (int)pl.lo2(c, G);
     if (n1 < 0 || n1 > kMaxU1 || n2 > kMaxU2) return false;
-    if ((size_t)n1 * pl.B1 + (size_t)n2 * pl.B2 > cap) return false;
+    if (rows_pieces_bytes(H, I, m, n1, n2) > cap) return false;
   }
   return true;
 }
 
-size_t rows_smem_bytes(int H, int I, int m_max) {
-  RPlan pl;
-  pl.init(m_max, H, I);
-  (void)pl;
-  return kSmemLimit;   // the piece area takes what the static part and the h blocks leave
-}
+size_t rows_smem_bytes(int, int, int) { return kSmemLimit; }   // the pieces take what is left
 
 }  // namespace
 

@@ -23,6 +23,7 @@
 // order) before applying the router weight. This fills the second round of SMs with half-length
 // tiles instead of leaving most of them idle while a few full-length tiles finish.
 #include <algorithm>
+#include <type_traits>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -55,8 +56,16 @@ struct __align__(1024) GStage {
   uint16_t sc[2][128];          // their scales, in row order
 };
 
+// Stage of the bf16-weight variant: one 64-wide K slice of the token rows and of both weight
+// blocks, all three as 128-byte-swizzled K-major tiles straight from TMA (MMA operands in place).
+struct __align__(1024) GStageBf {
+  uint8_t b[kBBoxBytes];        // token rows, K slice of 64 (SW128)
+  uint8_t a[2][kBBoxBytes];     // weight rows of block 0 and block 1, same K slice (SW128)
+};
+
+template <bool kBf16>
 struct GSmem {
-  GStage st[kGStages];
+  typename std::conditional<kBf16, GStageBf, GStage>::type st[kGStages];
   uint16_t ostage[128][256];    // epilogue: the tile's outputs, token-major (bf16, 64 KB)
   uint64_t full[kGStages], empty[kGStages];
   uint64_t afull[2], aempty[2];
@@ -100,6 +109,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(tc::smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(tc::smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;"
+      ::"r"(tc::smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(tc::smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -184,11 +202,17 @@ __device__ __forceinline__ TileDesc describe(const GParams& P, int32_t packed) {
   return d;
 }
 
+// kBf16: the weights are unquantised bf16 rows (the BF16 comparison configuration); a 2-D tensor
+// map brings each 128-row x 64-K slice of both blocks into shared memory in the MMA's operand
+// layout, the two issuers run tcgen05.mma with both operands in shared memory, and the
+// dequantiser warps stay idle. Tile scheduling, epilogue and combine are the W4 kernel's.
+template <bool kBf16>
 __global__ void __launch_bounds__(kGThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ BMaps xm) {
   extern __shared__ __align__(1024) uint8_t gsmem_raw[];
   // the dynamic shared window is only guaranteed 16-byte aligned: align the carve-out by hand
-  GSmem& s = *reinterpret_cast<GSmem*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
+  GSmem<kBf16>& s =
+      *reinterpret_cast<GSmem<kBf16>*>((reinterpret_cast<uintptr_t>(gsmem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -196,19 +220,19 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
   if (tid == 0) {
     for (int i = 0; i < kGStages; ++i) {
       tc::mbar_init(&s.full[i], 1);
-      tc::mbar_init(&s.empty[i], 8 + 2);       // 8 dequant warps + the two issuers' commits
+      tc::mbar_init(&s.empty[i], kBf16 ? 2 : 8 + 2);   // (8 dequant warps +) the two issuers' commits
     }
     for (int i = 0; i < 2; ++i) { tc::mbar_init(&s.afull[i], 8); tc::mbar_init(&s.aempty[i], 2); }
     tc::mbar_init(&s.dfull, 2);
     tc::mbar_init(&s.dempty, 4);
-    for (int i = 0; i < 4; ++i) { tc::mbar_init(&s.tq_full[i], 1); tc::mbar_init(&s.tq_empty[i], 2 + 4 + 8); }
+    for (int i = 0; i < 4; ++i) { tc::mbar_init(&s.tq_full[i], 1); tc::mbar_init(&s.tq_empty[i], kBf16 ? 2 + 4 : 2 + 4 + 8); }
     tc::mbar_init(&s.drain[0], 1);
     tc::mbar_init(&s.drain[1], 1);
     s.abort = 0;
     tc::fence_barrier_init();
     for (int i = 0; i < 3; ++i) asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.m[i]) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.wc) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.ws) : "memory");
+    if (!kBf16) asm volatile("prefetch.tensormap [%0];" ::"l"(&xm.ws) : "memory");
   }
   if (warp == 1) {
     tc::tmem_alloc<kGTmemCols>(&s.tmem_base);
@@ -248,6 +272,22 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
       const int z0 = d.slot * P.rg_slot + (int)d.rb0 * (kRowBlock / kRowGroup);
       const int z1 = d.slot * P.rg_slot + (int)d.rb1 * (kRowBlock / kRowGroup);
       bool ok = true;
+      if constexpr (kBf16) {
+        // 64-wide K slices; weight rows of block b at (slot * N + 128 * rb) of the bank's map
+        const int y0 = d.slot * P.rg_slot * kRowGroup + (int)d.rb0 * kRowBlock;
+        const int y1 = d.slot * P.rg_slot * kRowGroup + (int)d.rb1 * kRowBlock;
+        for (int ks = 2 * d.g0; ks < 2 * d.g1; ++ks, ++it) {
+          const int st = it % kGStages;
+          if (!gwait(&s.empty[st], ((it / kGStages) & 1) ^ 1, abort)) { ok = false; break; }
+          if (lane == 0) {
+            GStageBf& S = s.st[st];
+            tc::mbar_arrive_expect_tx(&s.full[st], bbytes + 2 * kBBoxBytes);
+            tma_load_2d(S.b, xmap, ks * 64, d.p0, &s.full[st]);
+            tma_load_2d_hint(S.a[0], &xm.wc, ks * 64, y0, &s.full[st], pol_w);
+            tma_load_2d_hint(S.a[1], &xm.wc, ks * 64, y1, &s.full[st], pol_w);
+          }
+        }
+      } else {
       for (int g = d.g0; g < d.g1; ++g, ++it) {
         const int st = it % kGStages;
         if (!gwait(&s.empty[st], ((it / kGStages) & 1) ^ 1, abort)) { ok = false; break; }
@@ -262,6 +302,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           tc::tma_load_3d(S.sc[1], &xm.ws, 0, g, z1, &s.full[st], pol_w);
           if (it < 16) gtrace(P, 48 + it);
         }
+      }
       }
       if (!ok) {
         if (lane == 0) report_status(P.ctl, MOE_ERR_TIMEOUT, 22);
@@ -298,6 +339,22 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
         tc::tc_fence_after();
         if (me == 0 && n == 1) gtrace(P, 3);
         bool ok = true;
+        if constexpr (kBf16) {
+          for (int ks = 2 * d.g0; ks < 2 * d.g1; ++ks, ++it) {
+            const int st = it % kGStages;
+            if (!tc::mbar_wait(&s.full[st], (it / kGStages) & 1, abort)) { ok = false; break; }
+            tc::tc_fence_after();
+            const uint32_t bbase = tc::smem_u32(s.st[st].b), abase = tc::smem_u32(s.st[st].a[me]);
+            const uint32_t dacc = tmem + (me ? kGD1 : kGD0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t adesc = tc::smem_desc(abase + kk * 32, 16, 1024, 2);
+              const uint64_t bdesc = tc::smem_desc(bbase + kk * 32, 16, 1024, 2);
+              tc::mma_ss(dacc, adesc, bdesc, idesc, (ks > 2 * d.g0 || kk > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(&s.empty[st]);
+          }
+        } else {
         for (int g = d.g0; g < d.g1; ++g, ++it, ++a_it) {
           const int st = it % kGStages, ab = a_it & 1;
           if (!tc::mbar_wait(&s.full[st], (it / kGStages) & 1, abort) ||
@@ -318,6 +375,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           tc::mma_commit(&s.empty[st]);
           if (me == 0 && a_it < 16) gtrace(P, 32 + a_it);
         }
+        }
         if (!ok) {
           report_status(P.ctl, MOE_ERR_TIMEOUT, 25);
           s.abort = 1;
@@ -332,6 +390,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
     __syncwarp();
   } else if (warp >= kGDq0 && warp < kGDq0 + 8) {
     // ---------------------------------------------------------------- dequantisers -> TMEM
+    if constexpr (!kBf16) {
     const int quarter = warp & 3, blk = (warp - kGDq0) >> 2;     // block 0 or 1 of the pair
     const int r = quarter * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16) + kGA + blk * 64;
@@ -386,6 +445,7 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
         if (warp == kGDq0 && lane == 0 && a_it < 16) gtrace(P, 16 + a_it);
       }
       if (!ok) break;
+    }
     }
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2..5)
@@ -606,12 +666,14 @@ int sm_count() {
   return g_sms;
 }
 
+template <bool kBf16>
 int launch_gemm(const GParams& P, const BMaps& map, int max_tiles, cudaStream_t s) {
-  const size_t smem = sizeof(GSmem) + 1024;
+  const size_t smem = sizeof(GSmem<kBf16>) + 1024;
   static bool attr = false;
   if (!attr) {
-    if (int rc = check_cuda(cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)smem), "grouped GEMM: smem attribute"))
+    if (int rc = check_cuda(cudaFuncSetAttribute(grouped_gemm_kernel<kBf16>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                            "grouped GEMM: smem attribute"))
       return rc;
     attr = true;
   }
@@ -625,7 +687,7 @@ int launch_gemm(const GParams& P, const BMaps& map, int max_tiles, cudaStream_t 
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel, P, map);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<kBf16>, P, map);
   note_launch();
   return check_cuda(e, "grouped_gemm_kernel launch");
 }
@@ -679,10 +741,19 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   }
 
   // the banks hold at least E slots' worth of addressable rows (slot indices are < E)
-  if (int rc = make_chunk_code_map(&xmap.wc, a.w13, 2 * a.I, a.H, a.E)) return rc;
-  if (int rc = make_chunk_scale_map(&xmap.ws, a.s13, 2 * a.I, a.H, a.E)) return rc;
-  if (int rc = make_chunk_code_map(&hmap.wc, a.w2, a.H, a.I, a.E)) return rc;
-  if (int rc = make_chunk_scale_map(&hmap.ws, a.s2, a.H, a.I, a.E)) return rc;
+  if (a.bf16_weights) {
+    // unquantised rows: [E * 2I][H] and [E * H][I] bf16, boxes of 128 rows x 64 K (128-byte swizzle)
+    if (int rc = make_rows_map(&xmap.wc, a.w13, a.E * 2 * a.I, a.H, kRowBlock)) return rc;
+    if (int rc = make_rows_map(&hmap.wc, a.w2, a.E * a.H, a.I, kRowBlock)) return rc;
+  } else {
+    if (int rc = make_chunk_code_map(&xmap.wc, a.w13, 2 * a.I, a.H, a.E)) return rc;
+    if (int rc = make_chunk_scale_map(&xmap.ws, a.s13, 2 * a.I, a.H, a.E)) return rc;
+    if (int rc = make_chunk_code_map(&hmap.wc, a.w2, a.H, a.I, a.E)) return rc;
+    if (int rc = make_chunk_scale_map(&hmap.ws, a.s2, a.H, a.I, a.E)) return rc;
+  }
+  auto gemm = [&](const GParams& Pg, const BMaps& m, int max_tiles) {
+    return a.bf16_weights ? launch_gemm<true>(Pg, m, max_tiles, s) : launch_gemm<false>(Pg, m, max_tiles, s);
+  };
 
   GParams P{};
   P.rg_slot = 2 * a.I / kRowGroup;
@@ -691,14 +762,14 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
   P.perm = perm; P.wts = a.wts; P.out = hp; P.out_ld = a.I; P.Tk = Tk; P.ctl = ctl;
   P.trace = nullptr;
-  if (int rc = launch_gemm(P, xmap, max_chunks * IB, s)) return rc;
+  if (int rc = gemm(P, xmap, max_chunks * IB)) return rc;
 
   P.rg_slot = a.H / kRowGroup;
   P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
   P.ksplit = ksplit; P.part_stride = ksplit == 2 ? (size_t)Tk * a.H : 0;   // the partials fill the fp32-sized yp
   P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;
   P.trace = dec::g_trace;
-  if (int rc = launch_gemm(P, hmap, max_chunks * HP * ksplit, s)) return rc;
+  if (int rc = gemm(P, hmap, max_chunks * HP * ksplit)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
   note_launch();
