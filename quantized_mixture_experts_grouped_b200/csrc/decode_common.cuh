@@ -98,6 +98,8 @@ struct RouteSmem {
   uint32_t tokbits[kMaxT][kMaxExperts / 32];
   int act[kMaxExperts];
   int sl[kMaxExperts];      // slot of act[j]
+  uint8_t ntok[kMaxExperts];            // tokens routed to act[j]
+  uint8_t tok[kMaxExperts][kMaxT];      // ... in ascending order (the expert's compact token list)
   int nact;
   int over;
 };
@@ -120,13 +122,11 @@ __device__ inline void route_token_n(RouteSmem& rs, const DecParams& P, int t, i
   const int E = P.E, k = P.k;
   const uint16_t* lt = P.logits + (size_t)t * E;
   uint32_t key[kPer];
-  if (lane == 0 && t == 0) trace_clk(P, 13);
 #pragma unroll
   for (int i = 0; i < kPer; ++i) {
     const int e = lane + 32 * i;
     key[i] = (e < E) ? route_key(lt[e], e) : 0u;
   }
-  if (t == 0 && __shfl_sync(kFull, key[0], 0) != 1u && lane == 0) trace_clk(P, 14);
   uint32_t mine[8];    // lane (j % 32) keeps the winning key of choice j in mine[j / 32]
 #pragma unroll
   for (int i = 0; i < 8; ++i) mine[i] = 0;
@@ -144,7 +144,6 @@ __device__ inline void route_token_n(RouteSmem& rs, const DecParams& P, int t, i
     for (int i = 0; i < 8; ++i)
       if ((j & 31) == lane && (j >> 5) == i) mine[i] = win;
   }
-  if (lane == 0 && t == 0) trace_clk(P, 15);
   auto logit_of = [](uint32_t w) {
     const uint32_t ord = w >> 16;
     return bf16_bits_to_float((ord & 0x8000u) ? (ord & 0x7fffu) : (~ord & 0xffffu));
@@ -222,6 +221,10 @@ __device__ inline void route_finish(RouteSmem& rs, const DecParams& P, int tid, 
       for (int i = 0; i < w; ++i) a += __popc(rs.present[i]);
       rs.act[a] = tid;
       rs.sl[a] = slot_of(P.slot, tid);
+      int n = 0;
+      for (int t = 0; t < P.T; ++t)
+        if ((rs.tokbits[t][w] >> (tid & 31)) & 1u) rs.tok[a][n++] = (uint8_t)t;
+      rs.ntok[a] = (uint8_t)n;
     }
   }
   if (tid == 0) {
@@ -431,6 +434,32 @@ __device__ __forceinline__ void encode_group(const float (&v)[4], uint8_t* hi, u
   if (lane == 0) {
     const int a = __float_as_int(mx * (1.f / 32639.f));
     *rec = make_int4(8 * sum0, a, 8 * sum1, a);
+  }
+}
+
+// The same encoding with lane l holding elements 4 l .. 4 l + 3 of the group in v[0..3] (one
+// 8-byte load per lane); the columns and the record are identical to encode_group's.
+__device__ __forceinline__ void encode_group_c(const float (&v)[4], uint8_t* hi, uint8_t* lo, int4* rec, int lane) {
+  float mx = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+  const float inv = mx > 0.f ? 32639.f / mx : 0.f;
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int iv = max(-32639, min(32639, __float2int_rn(v[i] * inv)));
+    const int h8 = (iv + 128) >> 8, l8 = iv - 256 * h8;
+    const int at = (lane >> 1) * 8 + 2 * i + (lane & 1);   // element 4 lane + i, permuted in its 8-group
+    hi[at] = (uint8_t)h8;
+    lo[at] = (uint8_t)l8;
+    sum += iv;
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(kFull, sum, o);   // lanes 0..15 / 16..31
+  const int sum1 = __shfl_sync(kFull, sum, 16);
+  if (lane == 0) {
+    const int a = __float_as_int(mx * (1.f / 32639.f));
+    *rec = make_int4(8 * sum, a, 8 * sum1, a);
   }
 }
 
