@@ -59,8 +59,9 @@ def lib():
         L.orc_moe_ffn_bf16.argtypes = [P, c.c_int, c.c_int, c.c_int, c.c_int, c.c_int, P, P,
                                        P, P, P, c.c_int, P, P, c.c_int]
         L.orc_slot_wave.argtypes = [c.c_int, c.c_int, P, P, P, P, P, P, P, P]
+        L.orc_slot_wave_capped.argtypes = [c.c_int, c.c_int, c.c_int, P, P, P, P, P, P, P, P, P]
         for f in ("orc_quantize", "orc_pack", "orc_unpack", "orc_dequant", "orc_route",
-                  "orc_permute", "orc_moe_ffn", "orc_moe_ffn_bf16", "orc_slot_wave"):
+                  "orc_permute", "orc_moe_ffn", "orc_moe_ffn_bf16", "orc_slot_wave", "orc_slot_wave_capped"):
             getattr(L, f).restype = c.c_int
         _lib = L
     return _lib
@@ -211,14 +212,18 @@ class SlotState:
         self.last_used = np.zeros(S, np.int64)
         self.clock = np.zeros(1, np.int64)
 
-    def wave(self, needed: np.ndarray):
-        """needed uint8 [E] (modified in place). Returns (wave_table [E], loads [(expert, slot)])."""
+    def wave(self, needed: np.ndarray, cap: int = None, protect: np.ndarray = None):
+        """needed uint8 [E] (modified in place); cap: most experts in the wave (default S);
+        protect: uint8 [S], nonzero = slot must not be overwritten. Returns (wave_table [E],
+        loads [(expert, slot)])."""
         assert needed.dtype == np.uint8 and needed.flags["C_CONTIGUOUS"]
         table = np.zeros(self.E, np.int32)
         le = np.zeros(self.S, np.int32)
         ls = np.zeros(self.S, np.int32)
         n = np.zeros(1, np.int32)
-        rc = lib().orc_slot_wave(self.E, self.S, _p(self.slot_expert), _p(self.last_used), _p(self.clock),
-                                 _p(needed), _p(table), _p(le), _p(ls), _p(n))
+        pr = None if protect is None else np.ascontiguousarray(protect, dtype=np.uint8)
+        rc = lib().orc_slot_wave_capped(self.E, self.S, self.S if cap is None else int(cap), _p(pr),
+                                        _p(self.slot_expert), _p(self.last_used), _p(self.clock), _p(needed),
+                                        _p(table), _p(le), _p(ls), _p(n))
         _check(rc, "slot_wave")
         return table, list(zip(le[: n[0]].tolist(), ls[: n[0]].tolist()))

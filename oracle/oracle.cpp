@@ -359,17 +359,21 @@ int orc_moe_ffn_bf16(const uint16_t* x, int T, int H, int I, int E, int k,
 // pages give no policy, so this is the plainest reading: least-recently-used replacement).
 // State: slot_expert[S] (-1 = free), last_used[S], *clock. needed[E] (0/1) marks the experts
 // that still have to run this step; on return the experts of this wave are cleared from it.
+// cap (1..S) bounds the experts of one wave; protect[S] (may be null) marks slots that must not
+// be overwritten in this wave (a wave still reading them).
 //   - hits = needed experts already resident, misses = the others, both in ascending id;
-//   - the wave is every hit plus the first S - |hits| misses (all of them if they fit);
+//   - the wave is the first min(cap, |hits|) hits plus the first cap - (hits taken) misses;
 //   - each miss of the wave, in ascending id, takes the lowest free slot, else evicts the
-//     slot with the smallest last_used whose expert is not in this wave (ties: lowest slot);
+//     slot with the smallest last_used (ties: lowest slot) that is not protected and whose
+//     expert is not needed (neither in this wave nor waiting for a later one);
 //   - every slot of the wave gets last_used = *clock, then *clock += 1.
+// With cap = S and no protected slot every hit is in the wave and this is plain LRU.
 // Outputs: wave_table[E] = slot of each expert in the wave, -1 for all others;
 // loads_expert/loads_slot[*n_loads] = the misses in load order.
-int orc_slot_wave(int E, int S, int32_t* slot_expert, int64_t* last_used, int64_t* clock,
-                  uint8_t* needed, int32_t* wave_table, int32_t* loads_expert, int32_t* loads_slot,
-                  int* n_loads) {
-  if (E <= 0 || S <= 0 || !slot_expert || !last_used || !clock || !needed || !wave_table ||
+int orc_slot_wave_capped(int E, int S, int cap, const uint8_t* protect, int32_t* slot_expert, int64_t* last_used,
+                         int64_t* clock, uint8_t* needed, int32_t* wave_table, int32_t* loads_expert,
+                         int32_t* loads_slot, int* n_loads) {
+  if (E <= 0 || S <= 0 || cap < 1 || cap > S || !slot_expert || !last_used || !clock || !needed || !wave_table ||
       !loads_expert || !loads_slot || !n_loads)
     return 1;
   std::vector<int> slot_of(E, -1);
@@ -381,9 +385,9 @@ int orc_slot_wave(int E, int S, int32_t* slot_expert, int64_t* last_used, int64_
     if (slot_of[e] >= 0) hits.push_back(e); else misses.push_back(e);
   }
   std::vector<char> in_wave(E, 0);
-  for (int e : hits) in_wave[e] = 1;
-  const int room = S - (int)hits.size();
-  const int n_new = std::min(room, (int)misses.size());
+  const int n_hit = std::min(cap, (int)hits.size());
+  for (int i = 0; i < n_hit; ++i) in_wave[hits[i]] = 1;
+  const int n_new = std::min(cap - n_hit, (int)misses.size());
   for (int i = 0; i < n_new; ++i) in_wave[misses[i]] = 1;
   *n_loads = 0;
   for (int i = 0; i < n_new; ++i) {
@@ -394,7 +398,8 @@ int orc_slot_wave(int E, int S, int32_t* slot_expert, int64_t* last_used, int64_
     if (pick < 0) {
       for (int s = 0; s < S; ++s) {
         const int old = slot_expert[s];
-        if (old >= 0 && in_wave[old]) continue;
+        if (old >= 0 && (in_wave[old] || needed[old])) continue;
+        if (protect && protect[s]) continue;
         if (pick < 0 || last_used[s] < last_used[pick]) pick = s;
       }
     }
@@ -415,6 +420,12 @@ int orc_slot_wave(int E, int S, int32_t* slot_expert, int64_t* last_used, int64_
   }
   *clock += 1;
   return 0;
+}
+
+int orc_slot_wave(int E, int S, int32_t* slot_expert, int64_t* last_used, int64_t* clock, uint8_t* needed,
+                  int32_t* wave_table, int32_t* loads_expert, int32_t* loads_slot, int* n_loads) {
+  return orc_slot_wave_capped(E, S, S, nullptr, slot_expert, last_used, clock, needed, wave_table, loads_expert,
+                              loads_slot, n_loads);
 }
 
 }  // extern "C"

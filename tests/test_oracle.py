@@ -410,6 +410,73 @@ def test_slot_waves_invariants_random():
         assert len(hits) <= S
 
 
+def test_slot_capped_hand_worked_sequence():
+    st = oracle.SlotState(6, 4)
+    needed = np.zeros(6, np.uint8)
+    for line in open(os.path.join(GOLDEN, "slot_lru_capped.txt")):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        head, table, loads = line.split("|")
+        words = head.split()[1:]
+        want = [int(v) for v in words[: words.index("p")]]
+        prot = np.zeros(4, np.uint8)
+        for v in words[words.index("p") + 1:]:
+            if v != "-":
+                prot[int(v)] = 1
+        if not needed.any():
+            needed[want] = 1
+        else:
+            assert sorted(np.flatnonzero(needed).tolist()) == want
+        got_table, got_loads = st.wave(needed, cap=2, protect=prot)
+        assert got_table.tolist() == [int(v) for v in table.split()], line
+        assert got_loads == [tuple(int(a) for a in l.split(":")) for l in loads.split()], line
+    assert not needed.any()
+
+
+@pytest.mark.parametrize("E,S", [(64, 16), (9, 3), (40, 2)])
+def test_slot_capped_waves_invariants_random(E, S):
+    """Waves of at most S // 2 experts, each protecting the slots of the wave before it: every
+    needed expert runs exactly once per step, no protected slot is written, an expert resident
+    at the start of its step is never loaded again in it, and cap = S with nothing protected is
+    the plain policy."""
+    g = np.random.default_rng(E + S)
+    cap = S // 2
+    st = oracle.SlotState(E, S)
+    plain, capped_as_plain = oracle.SlotState(E, S), oracle.SlotState(E, S)
+    for step in range(150):
+        want = g.choice(E, g.integers(1, min(E, 3 * S) + 1), replace=False)
+        needed = np.zeros(E, np.uint8)
+        needed[want] = 1
+        resident_before = set(st.slot_expert[st.slot_expert >= 0].tolist())
+        seen, loaded = set(), set()
+        prot = np.zeros(S, np.uint8)
+        while needed.any():
+            before = st.slot_expert.copy()
+            table, loads = st.wave(needed, cap=cap, protect=prot)
+            wave = set(np.flatnonzero(table >= 0).tolist())
+            assert 0 < len(wave) <= cap and not (wave & seen)
+            seen |= wave
+            for e, sl in loads:
+                assert not prot[sl]                       # protected slots keep their expert
+                assert e not in resident_before or e in loaded
+                loaded.add(e)
+            assert np.array_equal(st.slot_expert[prot == 1], before[prot == 1])
+            for e in wave:
+                assert st.slot_expert[table[e]] == e
+            prot = np.zeros(S, np.uint8)
+            prot[table[table >= 0]] = 1
+        assert seen == set(want.tolist())
+        assert not (loaded & resident_before)             # hits are never reloaded
+        n1, n2 = needed.copy(), needed.copy()
+        n1[want] = 1
+        n2[want] = 1
+        while n1.any():
+            t1, l1 = plain.wave(n1)
+            t2, l2 = capped_as_plain.wave(n2, cap=S, protect=np.zeros(S, np.uint8))
+            assert t1.tolist() == t2.tolist() and l1 == l2
+
+
 # ----------------------------------------------------------------------------- FFN on bf16 weights
 
 def test_ffn_bf16_weights_equal_w4_on_exactly_representable_weights():
