@@ -267,6 +267,17 @@ int slot_table_update(moe_slot_cache* cache, uint64_t* needed_mask,
                       int32_t* wave_table, int32_t* misses, int* n_misses,
                       moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded);
 
+/* slot_table_update with two more knobs: at most max_wave experts in the wave (0 = S; more
+ * than S is MOE_ERR_ARG), and protect (HOST, uint8 [S], may be NULL): nonzero marks a slot that
+ * this wave must not overwrite (a wave still reading it). The wave is then the first
+ * min(max_wave, hits) hits plus misses up to max_wave, both in ascending id, and a miss evicts
+ * the least recently used slot that is neither protected nor holding a needed expert (one
+ * waiting for a later wave included). slot_table_update is max_wave = 0, protect = NULL. */
+int slot_table_update_ex(moe_slot_cache* cache, uint64_t* needed_mask,
+                         int32_t* wave_table, int32_t* misses, int* n_misses,
+                         moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded,
+                         int max_wave, const uint8_t* protect);
+
 /* Testing aid for failure handling: the n-th next refill copy of this cache (0 = the next
  * one) reports failure as if cudaMemcpyAsync had returned an error; n = -1 turns it off. */
 void moe_slot_cache_fail_copy_after(moe_slot_cache* cache, int n);
@@ -281,9 +292,12 @@ int64_t moe_slot_cache_state(const moe_slot_cache* cache, int32_t* slot_expert, 
 
 /* Runs one whole slot-cache layer: routing (idx/wts on device), a device->host read of the
  * routed expert set (the one synchronisation of this path), then for every wave
- * slot_table_update + the FFN restricted to that wave's experts, accumulating in fp32; the
- * last wave writes out. wave_tables: device int32 [E * (ceil(E/S)+1)] scratch for the
- * per-wave tables. Returns the number of waves in *n_waves and the misses in *n_loads. */
+ * slot_table_update_ex + the FFN restricted to that wave's experts, accumulating in fp32; the
+ * last wave writes out. With S >= 2 a wave holds at most S/2 experts and protects the slots of
+ * the wave before it, so its refills overlap that wave's FFN (they wait only for the wave two
+ * back); with S = 1 every refill waits for the wave before. wave_tables: device int32
+ * [E * (ceil(E/S)+1)] scratch for the per-wave tables (reused in turn). Returns the number of
+ * waves in *n_waves and the misses in *n_loads. */
 int moe_slot_cache_layer(moe_slot_cache* cache,
                          const uint16_t* x_bf16, const uint16_t* logits_bf16, int T, int k,
                          int32_t* idx, float* wts, int32_t* wave_tables,

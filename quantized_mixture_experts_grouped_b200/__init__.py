@@ -64,6 +64,7 @@ def _load() -> ctypes.CDLL:
         "moe_slot_cache_fail_copy_after": ([P, I], None),
         "moe_slot_cache_dry_run": ([P, I], None),
         "slot_table_update": ([P, P, P, P, c.POINTER(I), P, P, P], I),
+        "slot_table_update_ex": ([P, P, P, P, c.POINTER(I), P, P, P, I, P], I),
         "moe_slot_cache_state": ([P, P, P], c.c_int64),
         "moe_slot_cache_layer": ([P, P, P, I, I, P, P, P, P, Z, P, I, P, P, c.POINTER(I), c.POINTER(I)], I),
     }

@@ -22,9 +22,10 @@ struct moe_slot_cache {
   std::vector<int32_t> slot_expert;                  // [S], -1 free
   std::vector<int64_t> last_used;                    // [S]
   int64_t clock = 0;
-  cudaEvent_t compute_done = nullptr;                // last FFN that read the pool
+  cudaEvent_t wave_done[2] = {nullptr, nullptr};    // FFN of the last even / odd wave done
   cudaEvent_t loaded = nullptr;
-  std::vector<int32_t> wave_tables;                  // host copies of every wave's table
+  int32_t* wave_tables = nullptr;                    // host copies of every wave's table, pinned
+                                                     // ([E + 1][E]: the uploads stay asynchronous)
   std::vector<int32_t> idx_host;
   int fail_copies_after = -1;                        // test hook: fail the n-th next copy
   bool dry_run = false;                              // test hook: plan and commit, copy nothing
@@ -59,11 +60,16 @@ cudaError_t refill_copy(moe_slot_cache* c, void* dst, const void* src, size_t by
 // The events that order refills against the FFN launches of moe_slot_cache_layer, created on
 // its first call (creating the cache itself makes no CUDA call).
 int ensure_events(moe_slot_cache* c) {
-  if (!c->compute_done)
-    if (int rc = check_cuda(cudaEventCreateWithFlags(&c->compute_done, cudaEventDisableTiming), "event create"))
-      return rc;
+  for (cudaEvent_t& e : c->wave_done)
+    if (!e)
+      if (int rc = check_cuda(cudaEventCreateWithFlags(&e, cudaEventDisableTiming), "event create")) return rc;
   if (!c->loaded)
     if (int rc = check_cuda(cudaEventCreateWithFlags(&c->loaded, cudaEventDisableTiming), "event create"))
+      return rc;
+  if (!c->wave_tables)
+    if (int rc = check_cuda(cudaHostAlloc(reinterpret_cast<void**>(&c->wave_tables),
+                                          sizeof(int32_t) * (size_t)c->E * (c->E + 1), cudaHostAllocDefault),
+                            "pinned wave tables"))
       return rc;
   return MOE_OK;
 }
@@ -93,14 +99,15 @@ MOE_API int moe_slot_cache_create(int E, int S, int H, int I, const uint8_t* ban
   c->s2_bytes = sizeof(uint16_t) * (size_t)H * (I / kGroup);
   c->slot_expert.assign(S, -1);
   c->last_used.assign(S, 0);
-  c->wave_tables.assign((size_t)E * (E + 1), -1);
   *out = c;
   return MOE_OK;
 }
 
 MOE_API void moe_slot_cache_destroy(moe_slot_cache* c) {
   if (!c) return;
-  if (c->compute_done) cudaEventDestroy(c->compute_done);
+  for (cudaEvent_t e : c->wave_done)
+    if (e) cudaEventDestroy(e);
+  if (c->wave_tables) cudaFreeHost(c->wave_tables);
   if (c->loaded) cudaEventDestroy(c->loaded);
   delete c;
 }
@@ -114,9 +121,18 @@ MOE_API int64_t moe_slot_cache_state(const moe_slot_cache* c, int32_t* slot_expe
 
 MOE_API int slot_table_update(moe_slot_cache* c, uint64_t* needed_mask, int32_t* wave_table, int32_t* misses,
                               int* n_misses, moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded) {
+  return slot_table_update_ex(c, needed_mask, wave_table, misses, n_misses, copy_stream, reuse_ok, loaded, 0,
+                              nullptr);
+}
+
+MOE_API int slot_table_update_ex(moe_slot_cache* c, uint64_t* needed_mask, int32_t* wave_table, int32_t* misses,
+                                 int* n_misses, moe_stream_t copy_stream, moe_event_t reuse_ok, moe_event_t loaded,
+                                 int max_wave, const uint8_t* protect) {
   if (!c || !needed_mask || !wave_table || !misses || !n_misses)
     return fail(MOE_ERR_ARG, "slot_table_update: null pointer");
   const int E = c->E, S = c->S;
+  const int cap = max_wave <= 0 ? S : max_wave;
+  if (cap > S) return fail(MOE_ERR_ARG, "slot_table_update: max_wave %d exceeds the %d slots", max_wave, S);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
   auto needed = [&](int e) { return (needed_mask[e >> 6] >> (e & 63)) & 1ull; };
   std::vector<int> slot_of(E, -1);
@@ -125,9 +141,11 @@ MOE_API int slot_table_update(moe_slot_cache* c, uint64_t* needed_mask, int32_t*
   std::vector<int> hits, miss;
   for (int e = 0; e < E; ++e)
     if (needed(e)) (slot_of[e] >= 0 ? hits : miss).push_back(e);
+  // the wave: the first min(cap, hits) hits, then misses up to cap, both in ascending id
   std::vector<char> in_wave(E, 0);
-  for (int e : hits) in_wave[e] = 1;
-  const int n_new = std::min(S - (int)hits.size(), (int)miss.size());
+  const int n_hit = std::min(cap, (int)hits.size());
+  for (int i = 0; i < n_hit; ++i) in_wave[hits[i]] = 1;
+  const int n_new = std::min(cap - n_hit, (int)miss.size());
   for (int i = 0; i < n_new; ++i) in_wave[miss[i]] = 1;
 
   // plan on a copy of the state so that a failed copy can leave the committed state alone
@@ -138,12 +156,14 @@ MOE_API int slot_table_update(moe_slot_cache* c, uint64_t* needed_mask, int32_t*
     int pick = -1;
     for (int s = 0; s < S && pick < 0; ++s)
       if (se[s] < 0) pick = s;
-    if (pick < 0)
+    if (pick < 0)   // least recently used, neither protected nor holding an expert still needed
       for (int s = 0; s < S; ++s) {
-        if (se[s] >= 0 && in_wave[se[s]]) continue;
+        if (se[s] >= 0 && (in_wave[se[s]] || needed(se[s]))) continue;
+        if (protect && protect[s]) continue;
         if (pick < 0 || c->last_used[s] < c->last_used[pick]) pick = s;
       }
-    if (pick < 0) return fail(MOE_ERR_ARG, "slot_table_update: no evictable slot (internal)");
+    if (pick < 0)
+      return fail(MOE_ERR_ARG, "slot_table_update: no evictable slot (protected slots and needed experts hold all)");
     if (se[pick] >= 0) slot_of[se[pick]] = -1;
     se[pick] = e;
     slot_of[e] = pick;
@@ -215,19 +235,32 @@ MOE_API int moe_slot_cache_layer(moe_slot_cache* c, const uint16_t* x, const uin
     if (e < 0 || e >= E) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: routed expert %d out of range", e);
     mask[e >> 6] |= 1ull << (e & 63);
   }
-  std::vector<int32_t> miss(c->S);
+  // Waves overlap their refills with the FFN of the wave before: with two or more slots a wave
+  // holds at most S/2 experts and may not overwrite the slots of the wave before it (still
+  // running), so its copies only wait for the wave two back. With one slot every refill waits
+  // for the wave before. The first wave waits for nothing: the host synchronised above, after
+  // every earlier kernel of this stream. The device tables are reused in turn: their uploads
+  // run on the compute stream, after the FFN that read the previous contents.
+  const int S = c->S;
+  const bool overlap = S >= 2;
+  const int cap = overlap ? S / 2 : S, n_dev_tables = (E + S - 1) / S + 1;
+  std::vector<int32_t> miss(S);
+  std::vector<uint8_t> prot(S, 0);
   int wave = 0;
   auto any = [&]() { return (mask[0] | mask[1] | mask[2] | mask[3]) != 0; };
   while (any()) {
-    if (wave > (E + c->S - 1) / c->S) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: too many waves (internal)");
-    int32_t* table_h = c->wave_tables.data() + (size_t)wave * E;
+    if (wave >= E) return fail(MOE_ERR_ARG, "moe_slot_cache_layer: too many waves (internal)");
+    int32_t* table_h = c->wave_tables + (size_t)wave * E;
     int nm = 0;
-    if (int rc = slot_table_update(c, mask, table_h, miss.data(), &nm, copy_stream,
-                                   reinterpret_cast<moe_event_t>(c->compute_done),
-                                   reinterpret_cast<moe_event_t>(c->loaded)))
+    cudaEvent_t reuse = nullptr;
+    if (overlap && wave >= 2) reuse = c->wave_done[wave & 1];
+    if (!overlap && wave >= 1) reuse = c->wave_done[(wave - 1) & 1];
+    if (int rc = slot_table_update_ex(c, mask, table_h, miss.data(), &nm, copy_stream,
+                                      reinterpret_cast<moe_event_t>(reuse), reinterpret_cast<moe_event_t>(c->loaded),
+                                      cap, overlap ? prot.data() : nullptr))
       return rc;
     *n_loads += nm;
-    int32_t* table_d = wave_tables + (size_t)wave * E;
+    int32_t* table_d = wave_tables + (size_t)(wave % n_dev_tables) * E;
     if (int rc = check_cuda(cudaMemcpyAsync(table_d, table_h, sizeof(int32_t) * E, cudaMemcpyHostToDevice, s),
                             "moe_slot_cache_layer: upload wave table"))
       return rc;
@@ -240,7 +273,10 @@ MOE_API int moe_slot_cache_layer(moe_slot_cache* c, const uint16_t* x, const uin
     if (int rc = moe_w4a16_ffn(x, T, c->H, c->I, E, k, idx, wts, c->pool_w13, c->pool_s13, c->pool_w2, c->pool_s2,
                                table_d, workspace, workspace_bytes, last ? out : nullptr, flags, stream))
       return rc;
-    if (int rc = check_cuda(cudaEventRecord(c->compute_done, s), "moe_slot_cache_layer: record")) return rc;
+    if (int rc = check_cuda(cudaEventRecord(c->wave_done[wave & 1], s), "moe_slot_cache_layer: record")) return rc;
+    std::fill(prot.begin(), prot.end(), 0);
+    for (int e = 0; e < E; ++e)
+      if (table_h[e] >= 0) prot[table_h[e]] = 1;
     ++wave;
   }
   *n_waves = wave;

@@ -73,6 +73,56 @@ def test_policy_matches_the_oracle(E, S, steps, seed):
     assert total_waves > steps      # some steps needed more than one wave
 
 
+def _update_ex(cache, mask, table, misses, cap, protect):
+    n = ctypes.c_int(0)
+    rc = q.lib.slot_table_update_ex(cache.handle, mask.ctypes.data_as(ctypes.c_void_p),
+                                    table.ctypes.data_as(ctypes.c_void_p), misses.ctypes.data_as(ctypes.c_void_p),
+                                    ctypes.byref(n), None, None, None, cap,
+                                    None if protect is None else protect.ctypes.data_as(ctypes.c_void_p))
+    if rc:
+        raise q.MoeError(rc, q.lib.moe_last_error_string().decode())
+    return n.value
+
+
+@pytest.mark.parametrize("E,S,steps,seed", [(64, 16, 120, 5), (9, 3, 80, 6), (40, 2, 60, 7)])
+def test_overlapped_waves_match_the_oracle(E, S, steps, seed):
+    """The schedule of moe_slot_cache_layer with two or more slots: waves of at most S // 2
+    experts, each protecting the slots of the wave before it in the step."""
+    g = np.random.default_rng(seed)
+    cache = _cache(E, S)
+    ref = oracle.SlotState(E, S)
+    table = np.zeros(E, np.int32)
+    misses = np.zeros(S, np.int32)
+    cap = S // 2
+    for _ in range(steps):
+        want = g.choice(E, int(g.integers(1, min(E, 3 * S) + 1)), replace=False)
+        needed = np.zeros(E, np.uint8)
+        needed[want] = 1
+        mask = _mask(needed)
+        prot = np.zeros(S, np.uint8)
+        while needed.any():
+            ref_table, ref_loads = ref.wave(needed, cap=cap, protect=prot)
+            n = _update_ex(cache, mask, table, misses, cap, prot)
+            np.testing.assert_array_equal(table, ref_table)
+            assert [(int(misses[i]), int(table[misses[i]])) for i in range(n)] == ref_loads
+            np.testing.assert_array_equal(_unmask(mask, E), needed)
+            se, lu, clock = cache.state()
+            np.testing.assert_array_equal(se, ref.slot_expert)
+            np.testing.assert_array_equal(lu, ref.last_used)
+            assert clock == ref.clock[0]
+            prot = np.zeros(S, np.uint8)
+            prot[table[table >= 0]] = 1
+
+
+def test_update_ex_rejects_a_cap_above_the_slots():
+    cache = _cache(8, 2)
+    mask = np.array([0b110], np.uint64)
+    with pytest.raises(q.MoeError) as ei:
+        _update_ex(cache, mask, np.zeros(8, np.int32), np.zeros(2, np.int32), 3, None)
+    assert ei.value.code == q.MOE_ERR_ARG
+    assert mask[0] == 0b110
+
+
 def test_failed_refill_commits_nothing():
     cache = _cache(8, 2)
     mask = np.array([0b00000110], np.uint64)        # experts 1 and 2
