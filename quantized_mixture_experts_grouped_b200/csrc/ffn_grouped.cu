@@ -3,7 +3,7 @@
 // through fused grouped MoE kernels).
 //
 // Launch sequence: permute (group pairs by expert) -> gather rows -> tile plan -> gate/up GEMM
-// with fused silu(g)*u -> down GEMM (bf16 rows per token-expert pair) -> router-weighted combine.
+// with fused silu(g)*u -> down GEMM (fp32 rows per token-expert pair) -> router-weighted combine.
 //
 // Both GEMMs are one persistent tcgen05 kernel (sm_100a). A CTA tile is a PAIR of 128-row
 // weight blocks (gate rows f..f+127 and the matching up rows, or two consecutive row blocks of
@@ -19,8 +19,8 @@
 // Tiles are claimed dynamically (atomic counter). Every wait is bounded.
 // Split K for the down GEMM: when the down tiles would fill the SMs only about once (few token
 // chunks, long K = I), each tile's K range is split in two halves that run as separate tiles and
-// write separate bf16 partial outputs; the combine adds the two partials of each row (in a fixed
-// order) before applying the router weight. This fills the second round of SMs with half-length
+// add their fp32 partial rows into the zeroed output rows (two terms: the sum does not depend on
+// which half comes first). This fills the second round of SMs with half-length
 // tiles instead of leaving most of them idle while a few full-length tiles finish.
 #include <algorithm>
 #include <type_traits>
@@ -84,7 +84,6 @@ struct GParams {
   int rows_half;                            // gate/up: I (up block offset); down: unused
   int mode;
   int ksplit;                               // down: K halves per tile (1 or 2); gate/up: 1
-  size_t part_stride;                       // elements between the partial outputs of the K halves
   const int32_t* tile_list;                 // packed tiles
   const int32_t* ntiles;                    // total tile count (device)
   const int32_t* offsets;                   // grouped pair offsets [E+1]
@@ -92,7 +91,8 @@ struct GParams {
   unsigned long long* trace;                // optional per-CTA clock stamps (diagnostics)
   const int32_t* perm;                      // pair id of grouped position
   const float* wts;                         // router weights [T*k] (applied by the combine)
-  uint16_t* out;                            // gate/up: Hp [Tk][I]; down: Yp [Tk][H] (unweighted)
+  uint16_t* out;                            // gate/up: Hp [Tk][I] (bf16)
+  float* y32;                               // down: Yp [Tk][H] (fp32, unweighted)
   int out_ld;                               // row length of out
   int Tk;
   int* ctl;
@@ -464,9 +464,10 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
       if (!bar_and(1, 128, gwait(&s.dfull, n & 1, abort))) break;
       tc::tc_fence_after();
       if (warp == kGEpi0 && lane == 0 && n == 0) gtrace(P, 1);
-      // the whole tile: tensor memory -> registers -> shared memory (token-major, bf16); the
-      // accumulators are released as soon as they are read, so the next tile's MMAs overlap the
-      // 16-byte coalesced stores of whole output rows below
+      // the whole tile: tensor memory -> registers, then gate/up: h to shared memory (token-major,
+      // bf16) for 16-byte coalesced stores of whole rows below; down: fp32 rows straight to global
+      // memory. The accumulators are released as soon as they are read, so the next tile's MMAs
+      // overlap the stores
       const int etid = tid - kGEpi0 * 32;
       for (int c0 = 0; c0 < d.ntok; c0 += 32) {
         uint32_t v0[32], v1[32];
@@ -482,10 +483,24 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
             s.ostage[c0 + j][r] = __bfloat16_as_ushort(__float2bfloat16_rn(__fdividef(g * u, 1.f + __expf(-g))));
           }
         } else {
+          // fp32 rows straight from the registers: for each token the warp's 32 lanes (rows)
+          // write 128 contiguous bytes of each of the two row blocks. With the K split both
+          // halves add into the zeroed row: 0 + a + b = 0 + b + a exactly, whichever comes first.
+          float* yp = P.y32 + (size_t)(d.p0 + c0) * P.out_ld + (size_t)d.rb0 * kRowBlock + r;
+          if (P.ksplit == 2) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            s.ostage[c0 + j][r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v0[j])));
-            s.ostage[c0 + j][kRowBlock + r] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v1[j])));
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < d.ntok) {
+                atomicAdd(yp + (size_t)j * P.out_ld, __uint_as_float(v0[j]));
+                atomicAdd(yp + (size_t)j * P.out_ld + kRowBlock, __uint_as_float(v1[j]));
+              }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (c0 + j < d.ntok) {
+                yp[(size_t)j * P.out_ld] = __uint_as_float(v0[j]);
+                yp[(size_t)j * P.out_ld + kRowBlock] = __uint_as_float(v1[j]);
+              }
           }
         }
       }
@@ -505,21 +520,6 @@ grouped_gemm_kernel(const __grid_constant__ GParams P, const __grid_constant__ B
           for (int m = 0; m < 4; ++m) {
             const int t = t0 + (etid >> 4) + 8 * m;
             if (t < d.ntok) *reinterpret_cast<uint4*>(P.out + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
-          }
-        }
-      } else {
-        // 256 columns = 32 pieces per token row; a warp stores one whole row per step (into the
-        // partial output of the tile's K half)
-        const size_t col = d.rb0 * kRowBlock + (etid & 31) * 8;
-        uint16_t* const outp = P.out + (size_t)d.part * P.part_stride;
-        for (int t0 = 0; t0 < d.ntok; t0 += 16) {
-          uint4 v[4];
-#pragma unroll
-          for (int m = 0; m < 4; ++m) v[m] = *reinterpret_cast<const uint4*>(&s.ostage[t0 + (etid >> 5) + 4 * m][(etid & 31) * 8]);
-#pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            const int t = t0 + (etid >> 5) + 4 * m;
-            if (t < d.ntok) *reinterpret_cast<uint4*>(outp + (size_t)(d.p0 + t) * P.out_ld + col) = v[m];
           }
         }
       }
@@ -569,15 +569,14 @@ __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t* __restric
   }
 }
 
-// out[t] = bf16( acc + sum_j wts[t][j] * y[inv[t][j]] ) over the bf16 down-projection rows y,
-// in fixed j order. With K split in two, y = y_0 + y_1 (the halves' partial rows, added first).
-__global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __restrict__ yw, size_t part_stride,
-                                                           const float* __restrict__ wts,
-                                                           const int32_t* __restrict__ idx,
-                                                           const int32_t* __restrict__ inv,
-                                                           const int32_t* __restrict__ table, int H, int k,
-                                                           float* __restrict__ acc, bool accumulate,
-                                                           uint16_t* __restrict__ out) {
+// out[t] = bf16( acc + sum_j wts[t][j] * y[inv[t][j]] ) over the fp32 down-projection rows y, in
+// fixed j order.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yp, const float* __restrict__ wts,
+                                                      const int32_t* __restrict__ idx,
+                                                      const int32_t* __restrict__ inv,
+                                                      const int32_t* __restrict__ table, int H, int k,
+                                                      float* __restrict__ acc, bool accumulate,
+                                                      uint16_t* __restrict__ out) {
   pdl_begin();
   const int t = blockIdx.x;
   const int n0 = (blockIdx.y * blockDim.x + threadIdx.x) * 8;
@@ -589,24 +588,9 @@ __global__ void __launch_bounds__(256) combine_bf16_kernel(const uint16_t* __res
   for (int j = 0; j < k; ++j) {
     if (slot_of(table, idx[(size_t)t * k + j]) < 0) continue;
     const float w = wts[(size_t)t * k + j];
-    const uint16_t* yrow = yw + (size_t)inv[(size_t)t * k + j] * H + n0;
-    const uint4 y = *reinterpret_cast<const uint4*>(yrow);
-    const uint32_t yy[4] = {y.x, y.y, y.z, y.w};
-    float yf[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      yf[2 * i] = bf16_bits_to_float(yy[i] & 0xffffu);
-      yf[2 * i + 1] = bf16_bits_to_float(yy[i] >> 16);
-    }
-    if (part_stride) {
-      const uint4 z = *reinterpret_cast<const uint4*>(yrow + part_stride);
-      const uint32_t zz[4] = {z.x, z.y, z.z, z.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        yf[2 * i] += bf16_bits_to_float(zz[i] & 0xffffu);
-        yf[2 * i + 1] += bf16_bits_to_float(zz[i] >> 16);
-      }
-    }
+    const float* yrow = yp + (size_t)inv[(size_t)t * k + j] * H + n0;
+    const float4 a0 = *reinterpret_cast<const float4*>(yrow), a1 = *reinterpret_cast<const float4*>(yrow + 4);
+    const float yf[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = fmaf(w, yf[i], v[i]);
   }
@@ -712,7 +696,6 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   int32_t* list_dn = list_gu + L.tile_list_len;
   uint16_t* xp = reinterpret_cast<uint16_t*>(a.ws + L.xp);
   uint16_t* hp = reinterpret_cast<uint16_t*>(a.ws + L.hp);
-  uint16_t* yw = reinterpret_cast<uint16_t*>(a.ws + L.yp);          // y per pair, bf16 (one or two K-half partials)
   int* ctl = reinterpret_cast<int*>(a.ws + L.status);
 
   if (int rc = launch_permute(a.idx, a.T, a.k, a.E, counts, offsets, perm, inv,
@@ -758,7 +741,7 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
   GParams P{};
   P.rg_slot = 2 * a.I / kRowGroup;
   P.K = a.H; P.G = a.H / kGroup; P.rows_half = a.I; P.mode = kModeGateUp;
-  P.ksplit = 1; P.part_stride = 0;
+  P.ksplit = 1;
   P.tile_list = list_gu; P.ntiles = tiles + 0; P.offsets = offsets; P.table = a.slot;
   P.perm = perm; P.wts = a.wts; P.out = hp; P.out_ld = a.I; P.Tk = Tk; P.ctl = ctl;
   P.trace = nullptr;
@@ -766,17 +749,22 @@ int ffn_grouped(const FfnArgs& a, cudaStream_t s) {
 
   P.rg_slot = a.H / kRowGroup;
   P.K = a.I; P.G = a.I / kGroup; P.rows_half = 0; P.mode = kModeDown;
-  P.ksplit = ksplit; P.part_stride = ksplit == 2 ? (size_t)Tk * a.H : 0;   // the partials fill the fp32-sized yp
-  P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = yw; P.out_ld = a.H;
+  // y per pair in fp32 (the one rounding left before the combine is the output's); with the K
+  // split both halves add into rows zeroed first
+  P.ksplit = ksplit;
+  P.tile_list = list_dn; P.ntiles = tiles + 1; P.out = nullptr; P.out_ld = a.H;
+  P.y32 = reinterpret_cast<float*>(a.ws + L.yp);                    // y per pair, fp32 [Tk][H]
   P.trace = dec::g_trace;
+  if (ksplit == 2)
+    if (int rc = check_cuda(cudaMemsetAsync(P.y32, 0, sizeof(float) * (size_t)Tk * a.H, s), "zero y")) return rc;
   if (int rc = gemm(P, hmap, max_chunks * HP * ksplit)) return rc;
 
   dim3 grid(a.T, ceil_div(a.H, 256 * 8));
   note_launch();
-  return check_cuda(launch_pdl(combine_bf16_kernel, grid, dim3(256), 0, s, (const uint16_t*)yw, P.part_stride, a.wts, a.idx,
+  return check_cuda(launch_pdl(combine_kernel, grid, dim3(256), 0, s, (const float*)P.y32, a.wts, a.idx,
                                (const int32_t*)inv, a.slot, a.H, a.k, reinterpret_cast<float*>(a.ws + L.acc),
                                a.accumulate, a.out),
-                    "combine_bf16_kernel");
+                    "combine_kernel");
 }
 
 }  // namespace moe
