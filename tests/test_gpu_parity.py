@@ -219,6 +219,24 @@ def test_ffn_edge_cases_small_batch(path):
     assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"edge small {path}")
 
 
+@pytest.mark.parametrize("path", ["decode", "grouped"])
+def test_ffn_experts_with_every_token_count_width(path):
+    """16 tokens, top-3 of 8, routed so that five experts take 16, 10, 6, 3 and 13 tokens and
+    three take none: on the batched decode kernel these are four, three, two, one and four MMA
+    blocks of compact tokens per tile, in both phases."""
+    wl = mi.Workload("widths", H=512, I=256, E=8, k=3, T=16)
+    g = np.random.default_rng(12)
+    l = g.standard_normal((wl.T, wl.E)).astype(np.float32)
+    chosen = [(0, 1, 4)] * 10 + [(0, 2, 3)] * 3 + [(0, 2, 4)] * 3
+    for t, es in enumerate(chosen):
+        l[t, list(es)] += 100.0
+    layer = Layer(wl, logits=mi.to_bf16_bits(l))
+    counts = np.bincount(layer.idx.ravel(), minlength=wl.E)
+    assert counts.tolist() == [16, 10, 6, 3, 13, 0, 0, 0]
+    out, _ = _run_ffn(layer, path)
+    assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"token-count widths {path}")
+
+
 @pytest.mark.parametrize("path", ["auto", "decode", "simple", "grouped", "sequential"])
 @pytest.mark.parametrize("T", [1, 5, 16, 300])
 def test_layer_call_routes_and_runs(path, T):
@@ -464,6 +482,39 @@ def test_workspace_reused_across_sizes_and_paths():
         assert q.moe_workspace_status(ws) == 0, (T, path)
         np.testing.assert_array_equal(idx.cpu().numpy(), layer.idx)
         assert_ffn_close(bf16_dev_to_f32(out), layer.oracle_out(), f"reused workspace T={T} {path}")
+
+
+@pytest.mark.parametrize("path", ["decode", "grouped"])
+def test_slot_cache_layer_after_a_failed_wave_is_clean(path):
+    """A refill that fails in the second wave ends the layer call with MOE_ERR_CUDA after the
+    first wave's FFN has written the workspace's fp32 accumulator. The next call on the same
+    workspace starts its first wave by storing into the accumulator, not adding to it, so its
+    output matches the oracle."""
+    wl = mi.Workload("cachefail_layer", H=256, I=128, E=8, k=2, T=3)
+    layer = Layer(wl, step=4)
+    assert len(np.unique(layer.idx)) >= 3          # at least three waves of one expert (S = 2)
+    S = 2
+    cache = _make_cache(wl, S, layer)
+    copy_stream = torch.cuda.Stream()
+    ws = _ws(wl.T, wl.H, wl.I, wl.E, wl.k)
+    wave_tables = torch.empty(wl.E * (wl.E // S + 2), dtype=torch.int32, device="cuda")
+    d = layer.to_device()
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((wl.T, wl.k), dtype=torch.float32, device="cuda")
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    cache.fail_copy_after(5)      # wave 1 (one expert, four copies) succeeds, wave 2's second copy fails
+    with pytest.raises(q.MoeError) as ei:
+        cache.layer(d["x"], d["logits"], wl.k, idx, wts, wave_tables, ws, out, path=q.PATHS[path],
+                    copy_stream=copy_stream)
+    assert ei.value.code == q.MOE_ERR_CUDA
+    torch.cuda.synchronize()
+    assert q.moe_workspace_status(ws) == 0
+    out2 = torch.full((wl.T, wl.H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    n_waves, _ = cache.layer(d["x"], d["logits"], wl.k, idx, wts, wave_tables, ws, out2, path=q.PATHS[path],
+                             copy_stream=copy_stream)
+    torch.cuda.synchronize()
+    assert n_waves >= 2 and q.moe_workspace_status(ws) == 0
+    assert_ffn_close(bf16_dev_to_f32(out2), layer.oracle_out(), f"slot cache after a failed wave {path}")
 
 
 def test_slot_table_update_refill_failure_is_reported():
