@@ -139,13 +139,13 @@ int moe_workspace_status(void* workspace, moe_stream_t stream, int* status);
  * configurable GPU-resident slot cache and fused grouped MoE kernels"):
  *   y_e(x) = W2_e . ( silu(W_gate_e . x) * (W_up_e . x) ),  silu(z) = z / (1 + exp(-z))
  *   out[t] = sum_{j<k} wts[t][j] * y_{idx[t][j]}(x_t)
- * with W = q * s dequantised from the packed banks. The tcgen05 paths multiply bf16 operands
- * (bf16(q * s), and h rounded to bf16) with fp32 accumulation; the grouped path rounds each
- * token-expert pair's down projection to bf16 (when it splits K in two, each half, the halves
- * then added in fp32) before the router-weighted combine; the default fused decode kernel
- * (T <= 16) multiplies the codes exactly with x and h held as 16-bit fixed point per
- * 128-element group (32 for h at T = 1; error <= max|group| / 65278), scales applied in fp32.
- * out is bf16.
+ * with W = q * s dequantised from the packed banks. The grouped tcgen05 path multiplies bf16
+ * operands (bf16(q * s), and h rounded to bf16) with fp32 accumulation and keeps each
+ * token-expert pair's down projection in fp32 until the router-weighted combine (when it splits
+ * K in two, both halves add into the zeroed row: the same sum in either order); the fused decode
+ * kernels (T <= 16) multiply the codes exactly with x and h held as 16-bit fixed point per
+ * 128-element group (8-feature blocks for h at T = 1; error <= max|group| / 65278), scales
+ * applied in fp32. out is bf16.
  *   x: bf16 [T][H]; idx, wts: the router's outputs [T][k].
  *   w13/s13: packed W13 ([2I][H]) per slot, w2/s2: packed W2 ([H][I]) per slot;
  *     slot stride = moe_packed_bytes / moe_scales_count of the matrix.
@@ -214,7 +214,7 @@ int moe_noalloc_status(moe_stream_t stream, int* status);
  *   w13_bf16: bf16 [slots][2I][H] ([W_gate; W_up] rows, row-major), w2_bf16: bf16 [slots][H][I];
  *   16-byte aligned. Everything else as moe_w4a16_ffn / moe_w4a16_layer (same workspace);
  *   flags: MOE_PATH_AUTO or MOE_PATH_GROUPED, optionally | MOE_FLAG_ACCUMULATE. The per-pair down
- * projection is rounded to bf16 before the combine, as on the W4A16 grouped path.
+ * projection stays fp32 until the combine, as on the W4A16 grouped path.
  * Errors: MOE_ERR_ARG, MOE_ERR_SHAPE (H not a multiple of 256, as on the grouped path),
  * MOE_ERR_CUDA. */
 int moe_bf16_ffn(const uint16_t* x_bf16, int T, int H, int I, int E, int k,

@@ -57,7 +57,7 @@ struct WsLayout {
   size_t tile_list_len;
   size_t xp;            // bf16 [T*k][H] gathered activations
   size_t hp;            // bf16 [T*k][I] SwiGLU intermediate
-  size_t yp;            // fp32 [T*k][H] per-pair down projection (grouped path: two bf16 [T*k][H] K-half partials)
+  size_t yp;            // fp32 [T*k][H] per-pair down projection (grouped and reference paths)
   size_t acc;           // fp32 [T][H] accumulator for slot-cache waves
   size_t seq;           // int32 [E][E] one-expert slot tables of the sequential path
   size_t dec;           // fused-decode scratch

@@ -1,6 +1,6 @@
-// Pieces shared by the two fused decode kernels (tensor-core and CUDA-core): in-kernel routing,
-// the byte-balanced split of the selected experts' packed tiles over the CTAs, the scratch
-// layout, and the deterministic cross-CTA reductions ("Every Expert Counts: ExactMoE for
+// Pieces of the fused decode kernels: in-kernel routing and the compact token lists, the
+// byte-balanced split of the selected experts' packed tiles over the CTAs (batched kernel), the
+// scratch and counter layout, and the deterministic cross-CTA reductions ("Every Expert Counts: ExactMoE for
 // Memory-Efficient W4A16 Inference", Abstract: every selected expert runs through fused grouped
 // MoE kernels; the router's top-k is unchanged).
 //

@@ -20,8 +20,11 @@
 //    and the group's a it is the group's contribution in fp32. The one approximation is
 //    |x - a v| <= a / 2 = max|x| / 65278 per element (bf16 rounding of a value near max|x| is up
 //    to 128 times larger).
-// One MMA consumes 512 weights; a 128 x 128 tile takes 32 of them (8 per SM sub-partition),
-// against about 16 FP32 instructions per 32 weights on the CUDA cores.
+// The B columns of a tile are its expert's compact token list (the tokens routed to it), four
+// tokens per MMA block, so an expert with n tokens costs ceil(n / 4) blocks, not T / 4. A compute
+// warp does all 128 K of 16 rows of half the tiles of a stage (four MMAs into one accumulator per
+// block), and the phase-2 h operands are copied into the activation area once phase 1 is over,
+// so the ring's stages hold only codes and scales.
 #include "decode_common.cuh"
 
 namespace moe {
@@ -36,7 +39,7 @@ constexpr int kMMaxStages = 6;
 constexpr int kColPad = 64;                // bytes after each operand column: hi and lo columns of a token in
                                            // opposite bank halves (conflict-free 16-byte B loads)
 constexpr int kHCol = kRowBlock + kColPad; // bytes per h column in a tile (128 K + pad)
-constexpr int kRedStride = kRowBlock + 8;  // floats per (half, token) row of the block sums
+constexpr int kRedStride = kRowBlock + 8;  // floats per (warp half, token) row of the block sums
 // h bytes per (expert, K group) with KCOLS B columns: the columns, then one 16-byte record per
 // token (two columns per token)
 template <int KCOLS>
@@ -57,10 +60,11 @@ struct __align__(128) MSmem {
   uint64_t full[kMMaxStages], empty[kMMaxStages], hfull[kMMaxStages];
   RouteSmem rs;
   uint64_t redfull[2], redempty[2];
-  float red[2][2][TT][kRedStride];     // per-half block sums (two buffers)
+  float red[2][2][TT][kRedStride];     // block sums [buffer][warp half][token][row] (two buffers)
   int abort;
-  // followed in dynamic shared memory by the activation columns [kCols][H + kColPad] (bytes),
-  // their group records [H/128][4 NB] x 16 B and the stage ring
+  // followed in dynamic shared memory by the activation area (phase 1: the columns
+  // [kCols][H + kColPad] bytes and their group records [H/128][4 NB] x 16 B; phase 2: the ring
+  // slots' h operands) and the stage ring (codes and scales)
 };
 
 // Compute warp cw works on rows r0 = 16 (cw % 8) + g and r0 + 8, all 128 K, of the tiles
