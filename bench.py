@@ -61,11 +61,23 @@ PROFILE_SOURCES = ["quantized_mixture_experts_grouped_b200/csrc/ffn_decode_rows.
                    "quantized_mixture_experts_grouped_b200/csrc/tc.cuh"]
 
 
+def code_of(text: str) -> str:
+    """C++/CUDA source without its comments and blank space: what the compiler sees of it (a
+    comment-only edit does not change the kernel the profile was taken of). String literals that
+    contain comment markers are not special-cased; the profiled sources have none."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
 def source_hash(files=None) -> str:
-    """First 16 hex digits of the SHA-256 of the profiled kernel's source files, in order."""
+    """First 16 hex digits of the SHA-256 of the profiled kernel's source files, in order, with
+    comments and blank space removed (code_of)."""
     import hashlib
     files = PROFILE_SOURCES if files is None else files
-    return hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in files)).hexdigest()[:16]
+    code = "\n".join(code_of(open(os.path.join(ROOT, f), encoding="utf-8").read()) for f in files)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def profiled_traffic():

@@ -1,6 +1,6 @@
 """Host-side pieces of bench.py that the reported numbers rest on (CPU only): the algorithmic
 bytes per expert, and the ncu traffic figure that is only reported while the profiled kernel's
-sources are unchanged."""
+code is unchanged."""
 import os
 import shutil
 import sys
@@ -21,6 +21,13 @@ def test_expert_bytes_match_the_packed_layout():
     assert bench.expert_bytes(H, I) == codes + scales == 3_244_032
 
 
+def test_code_of_drops_comments_and_blank_space():
+    a = "int f(int x) {  // doubles\n  return 2 * x;   /* twice */\n}\n\n"
+    b = "int f(int x) {\n return 2 * x;\n}"
+    assert bench.code_of(a) == bench.code_of(b)
+    assert bench.code_of(a) != bench.code_of(b.replace("2", "3"))
+
+
 def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
     import json
     # a record written for copies of the profiled sources is read back while they are unchanged
@@ -34,9 +41,13 @@ def test_profiled_traffic_follows_the_kernel_sources(tmp_path, monkeypatch):
     record.write_text(json.dumps({"source_hash": bench.source_hash(), "traffic_bytes_per_launch": 12345}))
     monkeypatch.setattr(bench, "PROFILE", str(record))
     assert bench.profiled_traffic() == 12345
-    # any change to a profiled source drops the figure
+    # a comment-only edit leaves the compiled kernel, and so the figure, as it was
     with open(copies[0], "a") as fh:
-        fh.write("\n// edited\n")
+        fh.write("\n// edited\n/* and a block\n comment */\n")
+    assert bench.profiled_traffic() == 12345
+    # any change to the code drops the figure
+    with open(copies[0], "a") as fh:
+        fh.write("\nstatic int edited = 1;\n")
     assert bench.profiled_traffic() is None
     # so does a missing record
     monkeypatch.setattr(bench, "PROFILE", str(tmp_path / "missing.json"))
