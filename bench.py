@@ -939,6 +939,8 @@ def main():
                     help="skip the prefill layer measured after the default decode workload")
     ap.add_argument("--layers", type=int, default=None,
                     help="fewer layers than the workload's (profiling runs only; the metric uses 16)")
+    ap.add_argument("--routing", default=None, choices=["normal", "zipf"],
+                    help="router logits: N(0,1) or Zipf(1.1) popularity + Gumbel (default: the workload's)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per step other than the workload's (ablations; the metric uses the default)")
     args = ap.parse_args()
@@ -950,6 +952,9 @@ def main():
     if args.tokens is not None:
         import dataclasses
         wl = dataclasses.replace(wl, T=max(1, args.tokens))
+    if args.routing is not None:
+        import dataclasses
+        wl = dataclasses.replace(wl, routing=args.routing)
     rank, world, local = dist_setup(args)
     try:
         if args.impl == "reference":
