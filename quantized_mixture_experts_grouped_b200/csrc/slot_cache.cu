@@ -24,6 +24,9 @@ struct moe_slot_cache {
   int64_t clock = 0;
   cudaEvent_t wave_done[2] = {nullptr, nullptr};    // FFN of the last even / odd wave done
   cudaEvent_t loaded = nullptr;
+  cudaStream_t copy2 = nullptr;                      // second refill stream (two copies in flight
+  cudaEvent_t fork = nullptr, join = nullptr;        // on the link), forked from and joined to the
+                                                     // caller's copy stream per wave
   int32_t* wave_tables = nullptr;                    // host copies of every wave's table, pinned
                                                      // ([E + 1][E]: the uploads stay asynchronous)
   std::vector<int32_t> idx_host;
@@ -108,6 +111,9 @@ MOE_API void moe_slot_cache_destroy(moe_slot_cache* c) {
   for (cudaEvent_t e : c->wave_done)
     if (e) cudaEventDestroy(e);
   if (c->wave_tables) cudaFreeHost(c->wave_tables);
+  if (c->fork) cudaEventDestroy(c->fork);
+  if (c->join) cudaEventDestroy(c->join);
+  if (c->copy2) cudaStreamDestroy(c->copy2);
   if (c->loaded) cudaEventDestroy(c->loaded);
   delete c;
 }
@@ -175,24 +181,49 @@ MOE_API int slot_table_update_ex(moe_slot_cache* c, uint64_t* needed_mask, int32
     if (int rc = check_cuda(cudaStreamWaitEvent(cs, reinterpret_cast<cudaEvent_t>(reuse_ok), 0),
                             "slot_table_update: wait for pool reuse"))
       return rc;
+  // Two refill streams keep two copies on the link at once. For this copy pattern one stream
+  // measured 39.0 GB/s and two 43.6 GB/s on one B200 machine (four no more than two); where one
+  // stream already reaches ~44 GB/s the second changes nothing. The second stream is forked
+  // from the copy stream (so it waits for everything the copy stream waits for) and joined back
+  // before `loaded`. Experts alternate between the two; the issue order of the copies is
+  // unchanged.
+  cudaStream_t cs2 = cs;
+  if (loads_e.size() >= 2 && !c->dry_run) {
+    if (!c->copy2) {
+      if (int rc = check_cuda(cudaStreamCreateWithFlags(&c->copy2, cudaStreamNonBlocking), "second refill stream"))
+        return rc;
+      if (int rc = check_cuda(cudaEventCreateWithFlags(&c->fork, cudaEventDisableTiming), "event create")) return rc;
+      if (int rc = check_cuda(cudaEventCreateWithFlags(&c->join, cudaEventDisableTiming), "event create")) return rc;
+    }
+    if (int rc = check_cuda(cudaEventRecord(c->fork, cs), "slot_table_update: fork")) return rc;
+    if (int rc = check_cuda(cudaStreamWaitEvent(c->copy2, c->fork, 0), "slot_table_update: fork")) return rc;
+    cs2 = c->copy2;
+  }
   for (size_t i = 0; i < loads_e.size(); ++i) {
     const size_t e = loads_e[i], s = loads_s[i];
-    cudaError_t err = refill_copy(c, c->pool_w13 + s * c->w13_bytes, c->bank_w13 + e * c->w13_bytes, c->w13_bytes, cs);
+    cudaStream_t st = (i & 1) ? cs2 : cs;
+    cudaError_t err = refill_copy(c, c->pool_w13 + s * c->w13_bytes, c->bank_w13 + e * c->w13_bytes, c->w13_bytes, st);
     if (err == cudaSuccess)
       err = refill_copy(c, reinterpret_cast<char*>(c->pool_s13) + s * c->s13_bytes,
-                        reinterpret_cast<const char*>(c->bank_s13) + e * c->s13_bytes, c->s13_bytes, cs);
+                        reinterpret_cast<const char*>(c->bank_s13) + e * c->s13_bytes, c->s13_bytes, st);
     if (err == cudaSuccess)
-      err = refill_copy(c, c->pool_w2 + s * c->w2_bytes, c->bank_w2 + e * c->w2_bytes, c->w2_bytes, cs);
+      err = refill_copy(c, c->pool_w2 + s * c->w2_bytes, c->bank_w2 + e * c->w2_bytes, c->w2_bytes, st);
     if (err == cudaSuccess)
       err = refill_copy(c, reinterpret_cast<char*>(c->pool_s2) + s * c->s2_bytes,
-                        reinterpret_cast<const char*>(c->bank_s2) + e * c->s2_bytes, c->s2_bytes, cs);
+                        reinterpret_cast<const char*>(c->bank_s2) + e * c->s2_bytes, c->s2_bytes, st);
     if (err != cudaSuccess) {
       // slots written so far no longer hold what the committed state says: mark them free
       for (size_t j = 0; j <= i; ++j) c->slot_expert[loads_s[j]] = -1;
       *n_misses = 0;
+      if (cs2 != cs && cudaEventRecord(c->join, cs2) == cudaSuccess)   // keep the copy stream after both
+        cudaStreamWaitEvent(cs, c->join, 0);
       return fail(MOE_ERR_CUDA, "slot_table_update: refill of expert %zu into slot %zu failed: %s", e, s,
                   cudaGetErrorString(err));
     }
+  }
+  if (cs2 != cs) {
+    if (int rc = check_cuda(cudaEventRecord(c->join, cs2), "slot_table_update: join")) return rc;
+    if (int rc = check_cuda(cudaStreamWaitEvent(cs, c->join, 0), "slot_table_update: join")) return rc;
   }
   if (loaded)
     if (int rc = check_cuda(cudaEventRecord(reinterpret_cast<cudaEvent_t>(loaded), cs), "slot_table_update: record"))
